@@ -1,0 +1,19 @@
+"""B200-native (sm_100a) block self-attention for the Granite-Speech NAR encoder.
+
+The compute lives in ``libnle.so`` (``csrc/``, C ABI declared in
+``include/nle.h``); :mod:`chunked_block_self_b200.nle` is a thin ctypes
+binding with the same function names.  The binding is imported lazily so
+that :mod:`chunked_block_self_b200.workloads` can be used without the CUDA
+library (for instance to draw inputs on a CPU-only host).
+"""
+__all__ = ["nle", "workloads"]
+
+
+def __getattr__(name):
+    if name in ("nle", "workloads"):
+        import importlib
+        return importlib.import_module(f"{__name__}.{name}")
+    from . import nle as _nle
+    if hasattr(_nle, name):
+        return getattr(_nle, name)
+    raise AttributeError(name)

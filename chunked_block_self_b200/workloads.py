@@ -1,0 +1,153 @@
+"""Seeded synthetic inputs shaped like the pages' workloads.
+
+This module is shared by the tests, the bench and the smoke check; it feeds
+both the CUDA path and the CPU oracle.  It holds no attention arithmetic:
+only utterance lengths, packed offsets (``cu_seqlens``) and bf16 tensors
+drawn from a seeded ``numpy.random.default_rng``.
+
+Recipe (all inputs synthetic; no audio, no trained weights):
+
+* lengths are drawn first from the config's length rule, then Q, K, V as
+  float32 N(0, 1) times the config's factor, rounded to bf16
+  round-to-nearest-even (torch's float32 -> bf16 conversion).
+* default seed = 1000 + config number.
+
+The five workloads stand in for the pages' ones by shape only:
+
+1. one utterance of 400 frames (8 s at 50 Hz), 8 heads x 64;
+2. the fixed 800-frame encoder bucket of the portable ONNX README, 16 x 64,
+   values N(0,1) * 0.5;
+3. 16 utterances of 39-94 s (1950-4700 frames, never a multiple of the
+   200-frame block, so each ends in a partial block), 16 x 64;
+4. 128 utterances of 2-16 s (100-800 frames), 16 x 64 -- the batch-128
+   throughput setting of the model card;
+5. the projector: 64 utterances of 4700 frames; K/V 16 x 64, three query
+   rows per 15-frame window.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    n_seq: int
+    t_min: int
+    t_max: int
+    heads: int
+    d_head: int
+    factor: float
+    block_frames: int = 200
+    avoid_multiple_of: int = 0      # redraw lengths divisible by this (0: never)
+    window_frames: int = 0          # > 0 for the windowed cross-attention
+    queries_per_window: int = 0
+
+
+CONFIGS = {
+    1: Workload("single utterance T=400, 8x64", 1, 400, 400, 8, 64, 1.0),
+    2: Workload("800-frame bucket, 16x64, x0.5", 1, 800, 800, 16, 64, 0.5),
+    3: Workload("16 utts 1950-4700 frames, 16x64", 16, 1950, 4700, 16, 64, 1.0,
+                avoid_multiple_of=200),
+    4: Workload("128 utts 100-800 frames, 16x64", 128, 100, 800, 16, 64, 1.0),
+    5: Workload("projector 64 x 4700 frames, 15-frame windows x 3 queries, 16x64",
+                64, 4700, 4700, 16, 64, 1.0, window_frames=15, queries_per_window=3),
+}
+
+
+def default_seed(cfg: int) -> int:
+    return 1000 + int(cfg)
+
+
+def draw_lengths(cfg: int, seed: int | None = None) -> np.ndarray:
+    """Utterance lengths in frames for config ``cfg`` (int64 numpy)."""
+    w = CONFIGS[cfg]
+    rng = np.random.default_rng(default_seed(cfg) if seed is None else seed)
+    out = np.empty(w.n_seq, np.int64)
+    for i in range(w.n_seq):
+        while True:
+            t = int(rng.integers(w.t_min, w.t_max + 1))
+            if not w.avoid_multiple_of or t % w.avoid_multiple_of:
+                break
+        out[i] = t
+    return out
+
+
+def cu_seqlens(lengths) -> np.ndarray:
+    """Packed offsets: int32 [n_seq + 1], cu[0] = 0, cu[i+1] = cu[i] + T_i."""
+    lengths = np.asarray(lengths, np.int64)
+    cu = np.zeros(len(lengths) + 1, np.int64)
+    np.cumsum(lengths, out=cu[1:])
+    if cu[-1] >= 2**31:
+        raise ValueError("total frames exceed int32")
+    return cu.astype(np.int32)
+
+
+def bf16_normal(rng: np.random.Generator, shape, factor: float = 1.0) -> torch.Tensor:
+    """float32 N(0,1) * factor from ``rng``, rounded to bf16 (CPU tensor)."""
+    x = rng.standard_normal(size=shape, dtype=np.float32)
+    if factor != 1.0:
+        x *= np.float32(factor)
+    return torch.from_numpy(x).to(torch.bfloat16)
+
+
+def block_inputs(cfg: int | None = None, seed: int | None = None, *, lengths=None,
+                 heads: int | None = None, d_head: int = 64, factor: float | None = None,
+                 block_frames: int | None = None) -> dict:
+    """Q, K, V (bf16 CPU, [total_frames, heads, d_head]) plus offsets.
+
+    Either a config number, or explicit ``lengths``/``heads`` for custom cases.
+    """
+    if cfg is not None:
+        w = CONFIGS[cfg]
+        seed = default_seed(cfg) if seed is None else seed
+        if lengths is None:
+            lengths = draw_lengths(cfg, seed)
+        heads = w.heads if heads is None else heads
+        d_head = w.d_head
+        factor = w.factor if factor is None else factor
+        block_frames = w.block_frames if block_frames is None else block_frames
+    lengths = np.asarray(lengths, np.int64)
+    heads = 1 if heads is None else heads
+    factor = 1.0 if factor is None else factor
+    block_frames = 200 if block_frames is None else block_frames
+    rng = np.random.default_rng(12345 if seed is None else seed + 7)
+    cu = cu_seqlens(lengths)
+    total = int(cu[-1])
+    q = bf16_normal(rng, (total, heads, d_head), factor)
+    k = bf16_normal(rng, (total, heads, d_head), factor)
+    v = bf16_normal(rng, (total, heads, d_head), factor)
+    return dict(q=q, k=k, v=v, cu=cu, lengths=lengths, heads=heads, d_head=d_head,
+                block_frames=block_frames, total=total)
+
+
+def window_inputs(n_query_rows: int, cfg: int | None = 5, seed: int | None = None, *,
+                  lengths=None, heads: int | None = None, d_head: int = 64,
+                  factor: float | None = None) -> dict:
+    """Inputs of the windowed cross-attention.
+
+    ``n_query_rows`` is the number of query rows the caller's window plan asks
+    for (this module does not cut windows).  K and V are [total_frames, heads,
+    d_head]; Q is [n_query_rows, heads, d_head]; all bf16 CPU tensors.
+    """
+    w = CONFIGS[cfg] if cfg is not None else None
+    if w is not None:
+        seed = default_seed(cfg) if seed is None else seed
+        if lengths is None:
+            lengths = draw_lengths(cfg, seed)
+        heads = w.heads if heads is None else heads
+        factor = w.factor if factor is None else factor
+    lengths = np.asarray(lengths, np.int64)
+    heads = 1 if heads is None else heads
+    factor = 1.0 if factor is None else factor
+    rng = np.random.default_rng(54321 if seed is None else seed + 11)
+    cu = cu_seqlens(lengths)
+    total = int(cu[-1])
+    k = bf16_normal(rng, (total, heads, d_head), factor)
+    v = bf16_normal(rng, (total, heads, d_head), factor)
+    q = bf16_normal(rng, (int(n_query_rows), heads, d_head), factor)
+    return dict(q=q, k=k, v=v, cu=cu, lengths=lengths, heads=heads, d_head=d_head,
+                total=total)

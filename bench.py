@@ -1,0 +1,429 @@
+"""Throughput of the hot path on B200: block self-attention + windowed
+cross-attention over one packed batch per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nle|reference]
+
+A step is one pass of the whole path over the batch-128 workload (128
+utterances of 100-800 frames, 16 heads x 64, the model card's batch-128
+throughput setting): the 200-frame block self-attention of the encoder and
+the projector's 15-frame / 3-query windowed cross-attention over the same
+utterances.  Inputs are synthetic (seeded N(0,1) bf16), resident in HBM
+before timing; they total ~0.75 GB, larger than the 126 MB L2, so L2 is not
+flushed between steps.  One JSON line is printed by rank 0.
+
+Multi-GPU (torchrun, one process per GPU): data-parallel replicas, each
+rank runs its own batch of the same shape (weak scaling); there is no
+collective on the data path.  Time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the test oracle, untuned) on the
+host cores for the same metric: each step is a bounded sample of (block,
+head) / (window, head) items of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from chunked_block_self_b200 import workloads as wl  # noqa: E402
+
+METRIC = "block-attn TFLOP/s & encoder frames/s on 1 B200; % of dense BF16 peak"
+CFG = 4
+B, W, QW, D = 200, 15, 3, 64
+
+# ncu DRAM traffic of the block-attention kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum), captured on the source whose hash is given; per
+# unit of algorithmic bytes, so it scales to any launch.  Reported only while
+# the kernel source is unchanged.
+NCU_TRAFFIC = {"source_sha256": None, "traffic_over_algorithmic": None}
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("block_attn_sm100a.cu", "nle_device.cuh"):
+        with open(os.path.join(ROOT, "chunked_block_self_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ work counts
+def block_work(lengths, heads):
+    """Algorithmic FLOPs and bytes of block attention (padding excluded)."""
+    s1 = s2 = 0
+    for t in lengths:
+        full, rem = divmod(int(t), B)
+        s1 += full * B + rem
+        s2 += full * B * B + rem * rem
+    flops = 4 * D * heads * s2            # QK^T and PV, 2 flops per MAC
+    bytes_ = 4 * 2 * D * heads * s1       # Q, K, V read + O written, bf16
+    return flops, bytes_
+
+
+def window_work(lengths, heads):
+    n_win = s1 = 0
+    for t in lengths:
+        nw = -(-int(t) // W)
+        n_win += nw
+        s1 += int(t)
+    flops = 4 * QW * D * heads * s1
+    bytes_ = 2 * D * heads * (2 * QW * n_win + 2 * s1)   # Q + O rows, K + V rows
+    return flops, bytes_, n_win
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls NVML (SM clock, clock-event reasons) while the timed region runs."""
+
+    NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+             0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(device_index)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that, no clocks
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self._nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = get_reasons(self._h)
+                for bit, name in self.NAMES.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if self._h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": getattr(self, "error", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_sample(lengths, q, k, v, cu, qw, kw, vw, heads, budget_s: float):
+    """Time the fp64 oracle on whole utterances of the workload, in order,
+    until `budget_s` seconds have passed.  Returns (flops, frames, seconds,
+    utterances, threads)."""
+    import oracle
+    flops = frames = 0
+    n_utt = 0
+    t0 = time.perf_counter()
+    qrow = 0
+    a = 0
+    while n_utt < len(lengths) and time.perf_counter() - t0 < budget_s:
+        t = int(lengths[n_utt])
+        local = np.array([0, t], np.int32)
+        oracle.block_attn(q[a:a + t], k[a:a + t], v[a:a + t], local, block_frames=B, n_threads=0)
+        nw = -(-t // W)
+        oracle.window_xattn(qw[qrow:qrow + QW * nw], kw[a:a + t], vw[a:a + t], local, W, QW, n_threads=0)
+        f1, _ = block_work([t], heads)
+        f2, _, _ = window_work([t], heads)
+        flops += f1 + f2
+        frames += t
+        a += t
+        qrow += QW * nw
+        n_utt += 1
+    return flops, frames, time.perf_counter() - t0, n_utt, oracle.threads_used(0)
+
+
+def cpu_info():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ------------------------------------------------------------------ arms
+def build_inputs(rank):
+    seed = wl.default_seed(CFG) + rank
+    x = wl.block_inputs(CFG, seed=seed)
+    lengths, heads = x["lengths"], x["heads"]
+    n_win = sum(-(-int(t) // W) for t in lengths)
+    y = wl.window_inputs(QW * n_win, cfg=None, lengths=lengths, heads=heads, seed=seed + 100)
+    return x, y
+
+
+def config_dict(x, n_win):
+    return {"workload": "batch-128: 128 utterances of 100-800 frames (2-16 s at 50 Hz), 16 heads x 64; "
+                        "200-frame block self-attention + 15-frame/3-query windowed cross-attention",
+            "n_seq": int(len(x["lengths"])), "total_frames": int(x["total"]), "heads": int(x["heads"]),
+            "d_head": D, "block_frames": B, "window_frames": W, "queries_per_window": QW,
+            "windows": int(n_win), "seed": wl.default_seed(CFG),
+            "l2": "inputs ~0.75 GB per rank > 126 MB L2; not flushed between steps",
+            "parallelism": "data-parallel replicas by utterance (no collective)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    x, y = build_inputs(0)
+    lengths, heads = x["lengths"], x["heads"]
+    n_win = sum(-(-int(t) // W) for t in lengths)
+    steps, warm = args.steps, args.warmup
+    budget = max(0.05, min(2.0, 90.0 / (steps + warm)))   # whole run stays within a few minutes
+    q, k, v, cu = x["q"], x["k"], x["v"], x["cu"]
+    for _ in range(warm):
+        oracle_sample(lengths, q, k, v, cu, y["q"], y["k"], y["v"], heads, budget)
+    tot_f = tot_fr = tot_t = 0.0
+    utts = 0
+    for _ in range(steps):
+        f, fr, t, nu, threads = oracle_sample(lengths, q, k, v, cu, y["q"], y["k"], y["v"], heads, budget)
+        tot_f += f
+        tot_fr += fr
+        tot_t += t
+        utts += nu
+    value = tot_f / tot_t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": warm, "ms_per_step": 1e3 * tot_t / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(x, n_win),
+            "frames_per_s": tot_fr / tot_t,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{utts} whole utterances over {steps} steps (block + window oracle, "
+                                       f"~{budget:.2f} s per step), {cpu_info()}"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_nle(args, rank, world, local):
+    from chunked_block_self_b200 import nle
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    x, y = build_inputs(rank)
+    lengths, heads = x["lengths"], x["heads"]
+    n_win = sum(-(-int(t) // W) for t in lengths)
+    assert nle.window_query_rows(x["cu"], W, QW) == QW * n_win
+    f_blk, by_blk = block_work(lengths, heads)
+    f_win, by_win, _ = window_work(lengths, heads)
+    flops_step = f_blk + f_win
+    frames_step = int(x["total"])
+
+    # device-resident inputs
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    cu = torch.from_numpy(x["cu"]).to(dev)
+    qw, kw, vw = (y[n].to(dev) for n in ("q", "k", "v"))
+    out = torch.empty_like(q)
+    ow = torch.empty_like(qw)
+    total = int(x["total"])
+    n_seq = len(lengths)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+
+    def step():
+        nle.nle_block_attn_fwd(q, k, v, out, cu, n_seq, total, heads, D, B, stream=sp)
+        nle.nle_window_xattn_fwd(qw, kw, vw, ow, cu, n_seq, total, QW * n_win, heads, D, W, QW, stream=sp)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K + 1)]
+    clocks = ClockSampler(local)
+    with clocks:
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        ev[0].record(stream)
+        for i in range(K):
+            nle.nle_block_attn_fwd(q, k, v, out, cu, n_seq, total, heads, D, B, stream=sp)
+            ev[2 * i + 1].record(stream)
+            nle.nle_window_xattn_fwd(qw, kw, vw, ow, cu, n_seq, total, QW * n_win, heads, D, W, QW, stream=sp)
+            ev[2 * i + 2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+    elapsed_ms = start.elapsed_time(end)
+    t_blk = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)) / K
+    t_win = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(K)) / K
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    ms_step = elapsed_ms / K
+
+    # ---- end to end through the public API: host (pinned) -> device, both
+    # kernels, device -> host of both outputs, every step
+    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+    hqw, hkw, hvw = (y[n].pin_memory() for n in ("q", "k", "v"))
+    hcu = torch.from_numpy(x["cu"]).pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    how = torch.empty(ow.shape, dtype=ow.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hqw, hkw, hvw, hcu))
+    d2h = hout.numel() * hout.element_size() + how.numel() * how.element_size()
+
+    def e2e_step():
+        for d_, h_ in ((q, hq), (k, hk), (v, hv), (qw, hqw), (kw, hkw), (vw, hvw), (cu, hcu)):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        how.copy_(ow, non_blocking=True)
+
+    ke = max(3, min(K, 20))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / ke
+    barrier(world)
+
+    # ---- CPU baseline: the oracle on the host cores, rank 0 at N=1 only
+    cpu_base = None
+    if world == 1 and not args.no_cpu_baseline:
+        f, fr, t, nu, threads = oracle_sample(lengths, x["q"], x["k"], x["v"], x["cu"], y["q"], y["k"], y["v"],
+                                              heads, args.cpu_seconds)
+        cpu_base = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                    "frames_per_s": fr / t,
+                    "sample": f"first {nu} of {n_seq} utterances ({fr} frames; block + window oracle, "
+                              f"{t:.1f} s, fp64, {threads} threads), {cpu_info()}"}
+
+    hbm_peak, tf_peak, tf_sust, peak_src = measured_peaks()
+    achieved_gbs = by_blk / (t_blk * 1e-3) / 1e9
+    traffic = None
+    if NCU_TRAFFIC["source_sha256"] == kernel_source_sha() and NCU_TRAFFIC["traffic_over_algorithmic"]:
+        traffic = NCU_TRAFFIC["traffic_over_algorithmic"] * by_blk
+    blk_tflops = f_blk / (t_blk * 1e-3) / 1e12
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": config_dict(x, n_win),
+        "frames_per_s": world * frames_step / (ms_step * 1e-3),
+        "pct_of_dense_bf16_peak": 100.0 * value / (world * tf_peak),
+        "block_attn": {"tflops": blk_tflops, "pct_of_dense_bf16_peak": 100.0 * blk_tflops / tf_peak,
+                       "achieved_gbs": achieved_gbs, "ms": t_blk, "frames_per_s": frames_step / (t_blk * 1e-3),
+                       "attainable_tflops": min(tf_peak, f_blk / by_blk * hbm_peak / 1e3),
+                       "ai_flop_per_byte": f_blk / by_blk},
+        "window_xattn": {"gbs": by_win / (t_win * 1e-3) / 1e9, "ms": t_win, "tflops": f_win / (t_win * 1e-3) / 1e12,
+                         "pct_of_hbm_peak": 100.0 * by_win / (t_win * 1e-3) / 1e9 / hbm_peak},
+        "roofline": {"kernel": "block_attn_kernel", "bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": achieved_gbs / hbm_peak, "traffic": traffic,
+                     "algorithmic_bytes": by_blk, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
+        "clocks": clocks.summary(),
+        "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke},
+        "gpu_launches": 2 * K,
+        "cpu_baseline": cpu_base,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["nle", "reference"], default="nle")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget (N=1 only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        return run_reference(args, rank, world)
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        return run_nle(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,391 @@
+// nle_device.cuh -- device primitives shared by the sm_100a kernels:
+// mbarrier + bounded waits, TMA / bulk copies, tcgen05 (TMEM alloc, MMA,
+// loads/stores), and the warp-level plan walker that maps a block (or
+// window) index of the packed batch to (utterance, first frame, length).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "nle.h"
+
+namespace nle {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+        "r"(bytes)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Record the first error of a launch.
+__device__ __forceinline__ void report(int32_t *status, int code)
+{
+    if (status)
+        atomicCAS(status, 0, code);
+}
+
+// Bounded wait for the phase with parity `parity` of barrier `bar`.
+// Called by all 32 lanes of a warp; the result is warp-uniform.  Returns
+// false if the CTA-wide abort flag was raised (by this or another warp) or
+// the wait exceeded limit_ns, in which case the abort flag is raised and
+// NLE_ERR_TIMEOUT recorded.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                         uint64_t limit_ns, int32_t *status)
+{
+    bool ok = mbar_try_wait(bar, parity);
+    if (!ok) {
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t it = 0;
+        while (!(ok = mbar_try_wait(bar, parity))) {
+            if ((++it & 31u) == 0) {
+                if (*abort_flag)
+                    break;
+                if (globaltimer_ns() - t0 > limit_ns) {
+                    *abort_flag = 1;
+                    report(status, NLE_ERR_TIMEOUT);
+                    break;
+                }
+            }
+        }
+    }
+    return __all_sync(kFull, ok);
+}
+
+// Bounded wait that ignores the abort flag (used while draining copies in
+// flight before the CTA exits).  Single thread.
+__device__ __forceinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > limit_ns)
+            return false;
+    return true;
+}
+
+// ---------------------------------------------------------------- copies
+__device__ __forceinline__ void tma_prefetch_desc(const void *tmap)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+// 2-D tiled TMA load (no multicast): box at (x, y) of `tmap` into smem `dst`,
+// completing transaction bytes on `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int32_t x, int32_t y,
+                                            uint32_t bar, uint64_t cache_policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar), "l"(cache_policy)
+        : "memory");
+}
+
+// Contiguous bulk copy global -> shared (no multicast); 16-byte aligned
+// addresses, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                          uint64_t cache_policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(cache_policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// Generic-proxy smem writes -> visible to the async proxy (TMA / tcgen05).
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- tcgen05
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16, one CTA.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16, one CTA.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 op issued so far by this thread
+// has completed.
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
+// lbo/sbo in bytes (multiples of 16).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
+// b_mn_major: B operand stored N-contiguous.  m in {64,128}, n % 16 == 0.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n, bool b_mn_major)
+{
+    return (1u << 4)                       // D = f32
+           | (1u << 7)                     // A = bf16
+           | (1u << 10)                    // B = bf16
+           | ((b_mn_major ? 1u : 0u) << 16) // B major
+           | ((n >> 3) << 17)              // N / 8
+           | ((m >> 4) << 24);             // M / 16
+}
+
+// 32 lanes x 32 columns of 32-bit TMEM -> registers (one lane per thread),
+// waiting for completion inside the same asm so the values are ready.
+#define NLE_R8(b) "=r"(r[b + 0]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), \
+                  "=r"(r[b + 5]), "=r"(r[b + 6]), "=r"(r[b + 7])
+__device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : NLE_R8(0), NLE_R8(8), NLE_R8(16), NLE_R8(24)
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : NLE_R8(0), NLE_R8(8)
+        : "r"(taddr)
+        : "memory");
+}
+#undef NLE_R8
+
+// 16 registers -> 32 lanes x 16 columns of TMEM (one lane per thread).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- math
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// ---------------------------------------------------------------- plan walker
+// Maps unit index u (a block of `unit` frames, or a window) of the packed
+// batch to its utterance, first frame and length.  Warp-cooperative: all 32
+// lanes call every method together and get warp-uniform results.  Looks at
+// 32 utterances at a time (their unit counts are prefix-summed across the
+// warp); queries must be non-decreasing, so one pass over cu_seqlens serves
+// a whole persistent-kernel loop.  An utterance whose offsets are negative,
+// decreasing or beyond total_frames contributes no units and is flagged.
+struct PlanWalker {
+    const int32_t *cu;
+    int n_seq;
+    int total;
+    int unit;
+    int base;       // first utterance of the current group of 32
+    int before;     // units in utterances [0, base)
+    int incl;       // this lane's inclusive prefix of units within the group
+    int start;      // cu[base + lane]
+    int len;        // frames of utterance base + lane (0 if invalid/absent)
+    int group_units;
+    int bad;        // warp-uniform: an invalid utterance was seen
+
+    __device__ __forceinline__ void load_group(int lane)
+    {
+        const int s = base + lane;
+        int a = 0, b = 0, n = 0, flag = 0;
+        if (s < n_seq) {
+            a = __ldg(cu + s);
+            b = __ldg(cu + s + 1);
+            if (a < 0 || b < a || b > total) {
+                flag = 1;
+                a = b = 0;
+            } else {
+                n = (b - a + unit - 1) / unit;
+            }
+        }
+        start = a;
+        len = b - a;
+        int x = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, x, o);
+            if (lane >= o)
+                x += y;
+        }
+        incl = x;
+        group_units = __shfl_sync(kFull, x, 31);
+        if (__any_sync(kFull, flag))
+            bad = 1;
+    }
+
+    __device__ __forceinline__ void init(const int32_t *cu_, int n_seq_, int total_, int unit_, int lane)
+    {
+        cu = cu_;
+        n_seq = n_seq_;
+        total = total_;
+        unit = unit_;
+        base = 0;
+        before = 0;
+        bad = 0;
+        load_group(lane);
+    }
+
+    // Locate unit u (>= every earlier query).  Returns false when u is past
+    // the last unit of the batch.
+    __device__ __forceinline__ bool find(long long u, int lane, int &frame0, int &L, int &seq)
+    {
+        while (u >= (long long)before + group_units) {
+            if (base + 32 >= n_seq)
+                return false;
+            before += group_units;
+            base += 32;
+            load_group(lane);
+        }
+        const int rel = (int)(u - before);
+        const unsigned m = __ballot_sync(kFull, (base + lane < n_seq) && incl > rel);
+        const int src = __ffs(m) - 1;
+        const int incl_s = __shfl_sync(kFull, incl, src);
+        const int st = __shfl_sync(kFull, start, src);
+        const int ln = __shfl_sync(kFull, len, src);
+        const int nb = (ln + unit - 1) / unit;
+        const int j = rel - (incl_s - nb);
+        frame0 = st + j * unit;
+        L = min(unit, ln - j * unit);
+        seq = base + src;
+        return true;
+    }
+};
+
+} // namespace nle

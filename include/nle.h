@@ -1,0 +1,194 @@
+/*
+ * nle.h -- C ABI of libnle.so: varlen block self-attention and windowed
+ * cross-attention on NVIDIA B200 (sm_100a).
+ *
+ * The operations (sources are the web pages this library follows):
+ *
+ *  Block self-attention -- granite-speech-4.1-2b-nar model card, "Model
+ *  Architecture", (1) CTC Speech Encoder: the encoder uses block attention
+ *  with 4-second audio blocks.  At 50 Hz encoder frames (100 Hz log-mel,
+ *  2-frame stacking) a block is 200 frames.  Utterances are packed back to
+ *  back ("Usage / Installation": sequence packing, is_causal=False).  Block j
+ *  of utterance i covers frames [cu[i] + j*B, cu[i] + min((j+1)*B, T_i)) with
+ *  T_i = cu[i+1] - cu[i]; every frame attends, bidirectionally, to every frame
+ *  of its block and to nothing else:
+ *      S = scale * Q_blk K_blk^T,  P = softmax_rows(S),  O_blk = P V_blk.
+ *
+ *  Windowed cross-attention -- same card, (2) Q-Former Projector: each
+ *  15-frame window is reduced to 3 queries via cross-attention.  Windows are
+ *  cut per utterance from its frame 0 like the blocks (the last one may be
+ *  partial); window g of the packed batch owns query rows
+ *  queries_per_window*g ... +queries_per_window-1, each attending to the
+ *  window's frames.
+ *
+ * Conventions for every entry point below:
+ *  - Tensor pointers (q, k, v, out, cu_seqlens, dev_status) are DEVICE
+ *    pointers owned by the caller.  The library never allocates, frees or
+ *    synchronises; every launch is asynchronous on `stream` (a cudaStream_t;
+ *    NULL = the legacy default stream).  Host-side table functions take HOST
+ *    pointers and say so.
+ *  - q, k, v, out hold bf16 values, row-major [rows][heads][d_head]: one row
+ *    per frame (or per query), heads next, d_head contiguous.  d_head must be
+ *    64.  Base pointers must be 16-byte aligned.
+ *  - cu_seqlens is int32 [n_seq + 1], cu[0] = 0, non-decreasing, cu[n_seq] =
+ *    total_frames.  The kernels read it on the device; a sequence whose
+ *    offsets fall outside [0, total_frames] or decrease is skipped (no output
+ *    is written for it) and, where a dev_status word is given, reported as
+ *    NLE_ERR_INVALID_ARG.  No access ever leaves the buffers described by
+ *    total_frames / n_query_rows.
+ *  - Softmax runs in fp32 with the scale folded into exp2; QK^T and PV
+ *    accumulate in fp32; P is rounded to bf16 before PV; out is rounded to
+ *    bf16 (round to nearest even).
+ *  - out must not alias q, k or v.
+ *  - Errors found on the host are returned before anything is launched:
+ *    NLE_ERR_INVALID_ARG, NLE_ERR_UNSUPPORTED, NLE_ERR_MISALIGNED.  A launch
+ *    failure returns NLE_ERR_CUDA.  n_seq == 0 or total_frames == 0 is a
+ *    successful no-op.
+ *  - Every wait inside a kernel is bounded.  Past the limit the kernel stores
+ *    NLE_ERR_TIMEOUT into *dev_status (when given), releases what it holds and
+ *    returns; the CUDA context stays usable.
+ */
+#ifndef NLE_H
+#define NLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NLE_ABI_VERSION 1
+
+typedef enum {
+    NLE_OK = 0,
+    NLE_ERR_INVALID_ARG = -1, /* null pointer with work to do, bad sizes    */
+    NLE_ERR_UNSUPPORTED = -2, /* d_head != 64, block_frames > 256, ...      */
+    NLE_ERR_MISALIGNED = -3,  /* pointer or row stride not 16-byte aligned  */
+    NLE_ERR_CUDA = -4,        /* launch or device-query failure             */
+    NLE_ERR_TIMEOUT = -5      /* a bounded in-kernel wait expired           */
+} nle_status;
+
+/* Flags for the _ex entry points. */
+#define NLE_FLAG_NONE 0
+/* Test hook: the load of the first work item is never issued, so its
+ * consumers' bounded waits expire and the kernel reports NLE_ERR_TIMEOUT.
+ * Exercises the timeout path without hanging the GPU. */
+#define NLE_FLAG_TEST_SKIP_FIRST_LOAD 1
+
+/* ABI version (NLE_ABI_VERSION of the build). */
+int nle_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *nle_status_string(int status);
+
+/* ---------------------------------------------------------------------
+ * Block self-attention (model card, "Model Architecture" (1)).
+ *
+ * q, k, v, out   device bf16 [total_frames][heads][64]
+ * cu_seqlens     device int32 [n_seq + 1]
+ * n_seq          number of packed utterances (>= 0)
+ * total_frames   rows of q/k/v/out; must equal cu[n_seq]; < 2^31
+ * heads          >= 1
+ * d_head         must be 64
+ * block_frames   frames per block, 1..256 (200 for 4 s at 50 Hz)
+ * stream         cudaStream_t
+ * Returns NLE_OK or a negative nle_status.
+ */
+int nle_block_attn_fwd(const void *q, const void *k, const void *v, void *out,
+                       const int32_t *cu_seqlens, int n_seq,
+                       int64_t total_frames, int heads, int d_head,
+                       int block_frames, void *stream);
+
+/* As nle_block_attn_fwd, plus:
+ * softmax_scale    <= 0 selects 1/sqrt(d_head)
+ * row_stride_qkv   elements between consecutive frames of q, k and v (for
+ *                  a fused QKV buffer); 0 selects heads*d_head; must be a
+ *                  multiple of 8 and >= heads*d_head.  out is always dense
+ *                  (row stride heads*d_head).
+ * dev_status       device int32 or NULL; receives the first in-kernel error
+ *                  (NLE_ERR_TIMEOUT or NLE_ERR_INVALID_ARG); never reset by
+ *                  the library.
+ * flags            NLE_FLAG_* (test hooks only; 0 in production)
+ * wait_limit_ns    limit of every in-kernel wait; 0 selects 1 s.
+ */
+int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v,
+                          void *out, const int32_t *cu_seqlens, int n_seq,
+                          int64_t total_frames, int heads, int d_head,
+                          int block_frames, float softmax_scale,
+                          int64_t row_stride_qkv, int32_t *dev_status,
+                          int flags, int64_t wait_limit_ns, void *stream);
+
+/* ---------------------------------------------------------------------
+ * Windowed cross-attention (model card, "Model Architecture" (2)).
+ *
+ * q, out          device bf16 [n_query_rows][heads][64]; n_query_rows must be
+ *                 queries_per_window * (number of windows), see
+ *                 nle_window_plan_host
+ * k, v            device bf16 [total_frames][heads][64]
+ * cu_seqlens_kv   device int32 [n_seq + 1] over the key/value frames
+ * window_frames   1..32 (15 on the pages)
+ * queries_per_window 1..8 (3 on the pages)
+ */
+int nle_window_xattn_fwd(const void *q, const void *k, const void *v,
+                         void *out, const int32_t *cu_seqlens_kv, int n_seq,
+                         int64_t total_frames, int64_t n_query_rows, int heads,
+                         int d_head, int window_frames,
+                         int queries_per_window, void *stream);
+
+/* As nle_window_xattn_fwd with an explicit scale (<= 0: 1/sqrt(d_head)),
+ * status word, test flags and wait limit (see nle_block_attn_fwd_ex). */
+int nle_window_xattn_fwd_ex(const void *q, const void *k, const void *v,
+                            void *out, const int32_t *cu_seqlens_kv, int n_seq,
+                            int64_t total_frames, int64_t n_query_rows,
+                            int heads, int d_head, int window_frames,
+                            int queries_per_window, float softmax_scale,
+                            int32_t *dev_status, int flags,
+                            int64_t wait_limit_ns, void *stream);
+
+/* ---------------------------------------------------------------------
+ * Block / window plans (the integer scheduling the kernels perform).
+ *
+ * nle_block_plan_host: HOST pointers.  Enumerates the blocks of the packed
+ * batch in order: out_seq[b] = utterance, out_j[b] = block index inside it,
+ * out_start[b] = first frame, out_len[b] = frames in the block.  Output
+ * arrays may be NULL to only count.  *n_blocks receives the count.
+ * Returns NLE_ERR_INVALID_ARG if cu is not non-decreasing from 0, or if the
+ * count exceeds capacity while arrays are given.
+ */
+int nle_block_plan_host(const int32_t *cu_host, int n_seq, int block_frames,
+                        int32_t *out_seq, int32_t *out_j, int32_t *out_start,
+                        int32_t *out_len, int capacity, int *n_blocks);
+
+/* The same table computed on the device by the walker the kernels use.
+ * cu_dev and the out_* arrays are DEVICE pointers (out_* may be NULL);
+ * n_blocks_dev (device int32, required) receives the total count; entries
+ * past `capacity` are not written.  Asynchronous on `stream`. */
+int nle_block_plan_dev(const int32_t *cu_dev, int n_seq, int64_t total_frames,
+                       int block_frames, int32_t *out_seq, int32_t *out_j,
+                       int32_t *out_start, int32_t *out_len, int capacity,
+                       int32_t *n_blocks_dev, void *stream);
+
+/* Window table on the host (HOST pointers): as nle_block_plan_host with
+ * window_frames, plus out_qrow[g] = queries_per_window * g.  *n_windows
+ * receives the count; the query tensor then has
+ * queries_per_window * (*n_windows) rows. */
+int nle_window_plan_host(const int32_t *cu_host, int n_seq, int window_frames,
+                         int queries_per_window, int32_t *out_seq,
+                         int32_t *out_w, int32_t *out_start, int32_t *out_len,
+                         int32_t *out_qrow, int capacity, int *n_windows);
+
+/* ---------------------------------------------------------------------
+ * Multi-GPU data parallelism (replicas by utterance; no collective on the
+ * data path).  HOST pointers.  Splits n_seq utterances of the given lengths
+ * into world_size contiguous shards balancing the attention cost
+ * sum over blocks of len^2.  out_bounds[r] .. out_bounds[r+1] is rank r's
+ * utterance range (out_bounds has world_size + 1 entries).
+ */
+int nle_shard_plan_host(const int32_t *lengths_host, int n_seq,
+                        int block_frames, int world_size, int32_t *out_bounds);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NLE_H */

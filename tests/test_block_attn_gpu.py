@@ -240,3 +240,18 @@ def test_timeout_path_reports_and_recovers(cuda_device):
     assert int(status.item()) == nle.NLE_ERR_TIMEOUT
     out2 = _run(x, cuda_device)
     _compare(out2, oracle.block_attn(x["q"], x["k"], x["v"], x["cu"]))
+
+
+@pytest.mark.parametrize("B,lengths", [(200, [200, 137]), (128, [128, 90]), (256, [250]), (64, [64, 40])])
+def test_running_max_rescale(B, lengths, cuda_device):
+    """Keys late in the row dominate, so the softmax's running maximum jumps by
+    more than its slack after earlier columns were written and the P already
+    written is rescaled (by an exact power of two)."""
+    x = wl.block_inputs(lengths=lengths, heads=2, seed=B + 1)
+    k = x["k"].float()
+    for a in np.cumsum([0] + lengths[:-1]):
+        hi = min(B, lengths[0]) - 4
+        k[a + hi - 3:a + hi] *= 12.0
+    x["k"] = k.to(torch.bfloat16)
+    out = _run(x, cuda_device, B=B)
+    _compare(out, oracle.block_attn(x["q"], x["k"], x["v"], x["cu"], block_frames=B))

@@ -13,24 +13,29 @@
 //               with 128-byte-swizzled TMA boxes (no multicast) into a ring
 //               of QK stages and a ring of two V stages; V lags QK by one
 //               item so Q/K run up to (stages) items ahead.
-//   warp 1      TMEM owner and MMA issuer (one elected lane):
-//                 S_t = Q_t K^T   tcgen05.mma kind::f16, M=128, N=NB (B
-//                                 rounded up to 16), K=64 in 4 steps
+//   warp 1      owns TMEM (allocates and frees it); warps 1-3 do no work.
+//   warps 4-7   tile slot 0 (block rows 0..127), warps 8-11 tile slot 1
+//               (rows 128..B-1, blocks longer than 128 frames).  The first
+//               warp of each warpgroup issues the slot's MMAs (one elected
+//               lane, warp-uniform descriptors):
+//                 S_t = Q_t K^T   tcgen05.mma kind::f16, M=128, N=ceil16(L),
+//                                 K=64 in 4 steps
 //                 O_t = P_t V     A operand = P in TMEM, B = V (N-major) in
-//                                 smem, M=128, N=64, K=NB in NB/16 steps
-//               t = 0 covers block rows 0..127, t = 1 rows 128..B-1.
-//               Before PV of a partial block it zeroes V rows L..ceil16(L)-1
-//               in shared memory (frames outside the block; P is 0 there,
-//               but 0 * Inf would be NaN).
-//   warps 2-3   idle (they complete warpgroup 0 for setmaxnreg).
-//   warps 4-7   softmax + epilogue of tile 0; warps 8-11 of tile 1.  Each
+//                                 smem, M=128, N=64, K=ceil16(L) in steps
+//                                 of 16
+//               Before PV of a partial block warpgroup 0 zeroes V rows
+//               L..ceil16(L)-1 in shared memory (frames outside the block;
+//               P is 0 there, but 0 * Inf would be NaN).  Each
 //               thread owns one block row (its TMEM lane) and reads S in
-//               register segments of up to 112 columns: segment max, p =
-//               exp2(S*scale*log2e - m) in fp32 with an integer running max m
-//               (keys >= L are 0 by index, never by value), row sum, bf16
-//               pack, P written back over S.  The epilogue reads O, divides by
-//               the row sum, rounds to bf16 and stores only rows < L with
-//               16-byte vector stores.
+//               64-column register segments: p = exp2(S*scale*log2e
+//               - m) in fp32 with one shift m per row (keys >= L are 0 by
+//               index, never by value), row sum, bf16 pack, P written back
+//               over S.  The epilogue reads O, divides by
+//               the row sum and rounds to bf16; a warp whose 32 rows all lie
+//               in the block stages them (128-byte swizzle) in shared memory
+//               and writes them with one TMA store, otherwise its rows < L are
+//               written with 16-byte vector stores.  Rows past the block end
+//               are never written.
 // The MMAs of an item stop at ceil16(L) keys, so a partial block costs only
 // its own keys.
 // TMEM (512 columns): tile slot t at column 256*t holds S (NB columns), then
@@ -44,30 +49,44 @@
 #include "nle_device.cuh"
 #include "nle_host.h"
 
+// Optional cycle trace of CTA 0 for performance analysis (not built by
+// default): NLE_TRACE_AT(role, item, event) stores clock64() into a device
+// buffer registered with nle_trace_set().
+#ifdef NLE_TRACE
+__device__ unsigned long long *g_nle_trace = nullptr;
+extern "C" int nle_trace_set(void *p)
+{
+    return cudaMemcpyToSymbol(g_nle_trace, &p, sizeof(p)) == cudaSuccess ? 0 : -1;
+}
+#define NLE_TRACE_AT(role, n, ev)                                                                       \
+    do {                                                                                                \
+        if (blockIdx.x == 0 && g_nle_trace && (n) < 64)                                                 \
+            g_nle_trace[((role) * 64 + (n)) * 16 + (ev)] = clock64();                                   \
+    } while (0)
+#else
+#define NLE_TRACE_AT(role, n, ev) \
+    do {                          \
+    } while (0)
+#endif
+
 namespace {
 
 using namespace nle;
 
-// Wide blocks (NB >= 176, the pages' 200-frame blocks among them) run three
-// warpgroups with a setmaxnreg split: warpgroup 0 (producer, MMA, two idle
-// warps) gives registers to the two softmax warpgroups, whose threads then
-// hold 112-column segments of S.  128 x 56 + 256 x 224 equals the launch
-// allocation 384 x 168; the host refuses to launch a build whose per-thread
-// count differs (a larger request would wait forever).  Narrower blocks run
-// ten warps without the split and 64-column segments.
-constexpr int kSplitMinNB = 176;
-constexpr int kRegsLaunch = 168;
-constexpr int kRegsLow = 56;
-constexpr int kRegsHigh = 224;
-static_assert(128 * kRegsLow + 256 * kRegsHigh == 384 * kRegsLaunch, "register split must match launch");
+// Three warpgroups: warp 0 producer, warp 1 TMEM owner, warps 2-3 idle,
+// warps 4-11 the two tile warpgroups (168 registers each; the softmax works
+// on 64-column segments of S).
+// The two tile warpgroups may take turns on the softmax (a token passed
+// through shared memory); by default they overlap, which keeps two softmax
+// warps per SM sub-partition and measured faster.
+#ifndef NLE_PINGPONG
+#define NLE_PINGPONG 0
+#endif
+constexpr bool kPingPong = NLE_PINGPONG != 0;
+constexpr int kThreads = 384;
+constexpr int kSoftmax0 = 4;
+constexpr int kSeg = 64;
 
-template <int NB>
-struct Shape {
-    static constexpr bool split = NB >= kSplitMinNB;
-    static constexpr int threads = split ? 384 : 320;
-    static constexpr int first_softmax_warp = split ? 4 : 2;
-    static constexpr int seg = split ? 112 : 64;
-};
 constexpr int kQTile = 128;        // MMA M (rows per tile)
 constexpr int kRowBytes = 128;     // one frame of one head: 64 bf16
 constexpr int kMaxQK = 4;          // QK ring depth upper bound
@@ -78,16 +97,18 @@ constexpr uint32_t kOCol = 128;     // O offset inside a tile slot
 
 struct Bars {
     uint64_t qk_full[kMaxQK];
-    uint64_t qk_empty[kMaxQK];
+    uint64_t qk_empty[kMaxQK];   // 2 arrivals: the two tile warpgroups
     uint64_t v_full[kSV];
-    uint64_t v_empty[kSV];
+    uint64_t v_ready[kSV];       // tail rows of a partial block zeroed
+    uint64_t v_empty[kSV];       // 2 arrivals: the two tile warpgroups
     uint64_t s_full[2];
-    uint64_t p_full[2];
+    uint64_t wg_p[2];            // 4 arrivals: P of the tile written
     uint64_t o_full[2];
-    uint64_t tmem_free[2];
-    uint64_t mma_done;
+    uint64_t wg_o[2];            // 4 arrivals: O of the tile read from TMEM
+    uint64_t mma_done[2];
     uint32_t tmem_base;
     int abort_flag;
+    int turn;                    // softmax phases completed (ping-pong token)
 };
 
 struct Params {
@@ -102,6 +123,8 @@ struct Params {
     uint32_t q_bytes;   // Q region of a QK stage
     uint32_t qk_bytes;  // QK stage
     uint32_t v_bytes;   // V stage
+    uint32_t stage_off; // output staging: stage_bufs x 4 KB per softmax warp
+    int stage_bufs;     // 2 (alternating) when shared memory allows, else 1
     float scale_log2;
     __nv_bfloat16 *out;
     int out_stride;     // elements between output frames (heads * 64)
@@ -112,25 +135,37 @@ struct Params {
 
 // Softmax of one TMEM lane quarter of a tile (32 rows, one per lane).
 //
-// S is read from TMEM in register segments of at most kSeg columns (a
-// multiple of 16, so each segment's P covers whole PV K-steps).  The running
-// maximum is kept as an integer m in the log2 domain (x = s * scale * log2e,
-// m = ceil(max x)), so p = exp2(x - m) <= 1 for the segment that set m.  A
-// later segment whose own max exceeds m by at most kSlack keeps m (its p
-// may reach 2^kSlack, harmless in fp32 / bf16); otherwise m moves up and the
-// P already written is rescaled by 2^(m_old - m_new), an exact power of two.
-// The result is the same softmax: every p of a row shares one m.
-constexpr float kSlack = 8.f;
+// In the log2 domain (x = s * scale * log2e) every p of a row is
+// exp2(x - m) for one shift m per row; softmax does not depend on m, which
+// only has to keep p in range.  m starts as the max of the row's first 16
+// keys, so the row's largest p is usually a small power above 1 (and exactly
+// 1 for a one-key block).  While p is formed, the largest exponent x - m of
+// the segment is tracked next to the exp; if any lane sees one above kYMax
+// (or a NaN), the warp takes the rare path: m moves up by a whole number k so
+// that the segment's max maps to 0, the segment is recomputed from the
+// registers that still hold it, and the P already written are rescaled by
+// 2^-k, an exact power of two.
+//
+// S is read from TMEM in register segments of SEG columns (a multiple of
+// 16, so each segment's P covers whole PV K-steps); each segment's exps are
+// one straight-line block.  P (bf16 pairs) is written back over S's first
+// columns.
+constexpr float kYMax = 32.f;
 
-template <int W>
-__device__ __forceinline__ void seg_load(uint32_t taddr, uint32_t (&s)[W])
+template <int W, int N>
+__device__ __forceinline__ void seg_issue(uint32_t taddr, uint32_t (&s)[N])
 {
+    static_assert(W <= N && W % 16 == 0, "segment width");
 #pragma unroll
     for (int c = 0; c + 32 <= W; c += 32)
         tmem_ld32_nowait(taddr + c, &s[c]);
     if constexpr (W % 32 == 16)
         tmem_ld16_nowait(taddr + W - 16, &s[W - 16]);
-    tmem_wait_ld();
+}
+
+template <int W, int N>
+__device__ __forceinline__ void seg_fence(uint32_t (&s)[N])
+{
 #pragma unroll
     for (int i = 0; i < W; ++i)
         reg_fence(s[i]);
@@ -148,59 +183,60 @@ __device__ __forceinline__ void seg_store(uint32_t taddr, const uint32_t (&pk)[W
         tmem_st8p(taddr + W / 2 - 8, &pk[W / 2 - 8]);
 }
 
-// Masks keys >= L (by index) to -inf and returns the segment's max.
-template <int W>
-__device__ __forceinline__ float seg_mask_max(uint32_t (&s)[W], int c0, int L)
+// Keys >= L (by index) -> -inf, branch-free (selects); only called for the
+// segment that holds L.
+template <int W, int N>
+__device__ __forceinline__ void seg_mask(uint32_t (&s)[N], int c0, int L)
 {
 #pragma unroll
-    for (int g = 0; g < W / 8; ++g) {
-        if (c0 + 8 * g + 8 > L) {   // warp-uniform
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if (c0 + 8 * g + e >= L)
-                    s[8 * g + e] = __float_as_uint(-INFINITY);
-        }
-    }
+    for (int i = 0; i < W; ++i)
+        s[i] = c0 + i < L ? s[i] : __float_as_uint(-INFINITY);
+}
+
+// Exact max of the first W values (rare path and the initial shift).
+template <int W, int N>
+__device__ __forceinline__ float seg_max(const uint32_t (&s)[N])
+{
     float mx[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e)
-        mx[e] = __uint_as_float(s[e]);
+        mx[e] = fmaxf(__uint_as_float(s[e]), __uint_as_float(s[8 + e]));
 #pragma unroll
-    for (int i = 8; i < W; ++i)
-        mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(s[i]));
-    return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    for (int i = 16; i + 16 <= W; i += 16)
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            mx[e] = fmax3(mx[e], __uint_as_float(s[i + e]), __uint_as_float(s[i + 8 + e]));
+    return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
-// p = exp2(s * sl2 - m) for keys < L (0 beyond), summed into l, packed to
-// bf16 pairs.
-template <int W>
-__device__ __forceinline__ void seg_exp(const uint32_t (&s)[W], uint32_t (&pk)[W / 2], int c0, int L, float sl2,
-                                        float m, float &l)
+// p = exp2(s * sl2 - m) for the W keys (masked keys hold -inf -> 0), packed
+// to bf16 pairs; returns the segment sum, and the largest exponent in ymax.
+// Straight-line code: one basic block per segment keeps the exps of the
+// whole segment in flight.
+template <int W, int N>
+__device__ __forceinline__ float seg_exp(const uint32_t (&s)[N], uint32_t (&pk)[W / 2], float sl2, float m,
+                                         float &ymax)
 {
     float ls[4] = {0.f, 0.f, 0.f, 0.f};
+    float ym[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int g = 0; g < W / 8; ++g) {
-        if (c0 + 8 * g < L) {   // warp-uniform; masked keys hold -inf -> 0
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float a = ex2_approx(fmaf(__uint_as_float(s[8 * g + 2 * e]), sl2, -m));
-                const float b = ex2_approx(fmaf(__uint_as_float(s[8 * g + 2 * e + 1]), sl2, -m));
-                ls[e] += a + b;
-                pk[4 * g + e] = pack_bf16x2(a, b);
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                pk[4 * g + e] = 0u;
-        }
+    for (int j = 0; j < W / 2; ++j) {
+        const float ya = fmaf(__uint_as_float(s[2 * j]), sl2, -m);
+        const float yb = fmaf(__uint_as_float(s[2 * j + 1]), sl2, -m);
+        ym[j & 3] = fmax3(ym[j & 3], ya, yb);
+        const float a = ex2_approx(ya);
+        const float b = ex2_approx(yb);
+        ls[j & 3] += a + b;
+        pk[j] = pack_bf16x2(a, b);
     }
-    l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+    ymax = fmaxf(fmaxf(ym[0], ym[1]), fmaxf(ym[2], ym[3]));
+    return (ls[0] + ls[1]) + (ls[2] + ls[3]);
 }
 
 // Multiply the bf16 P already in TMEM columns [0, ncols) by f, a power of
 // two <= 1 (exact up to underflow); lanes with f = 1 rewrite P unchanged.
 // Rare path; must be entered by the whole warp.
-__device__ __noinline__ void rescale_p(uint32_t tS, int ncols, float f)
+__device__ __forceinline__ void rescale_p(uint32_t tS, int ncols, float f)
 {
     tmem_wait_st();
     for (int c = 0; c < ncols; c += 8) {
@@ -220,73 +256,132 @@ __device__ __noinline__ void rescale_p(uint32_t tS, int ncols, float f)
     }
 }
 
-template <int C0, int W>
-__device__ __forceinline__ void softmax_segment(uint32_t tS, int L, float sl2, float &m, float &l)
+// Rare path of one segment (whole warp): S of the segment is still intact
+// in TMEM (its P has not been stored yet), so it is streamed again in
+// 16-column chunks: first its max, then m moves up by a whole k so that max
+// maps to <= 0, the segment's P is recomputed and stored, and the P already
+// written (columns < C0/2) are rescaled by 2^-k.  A chunk's P (columns
+// (C0+c)/2..+8) only overwrites S columns that have already been read.
+template <int W>
+__device__ __forceinline__ void softmax_rare(uint32_t tS, int C0, int L, float sl2, float &m, float &l)
 {
-    uint32_t s[W];
-    seg_load<W>(tS + C0, s);
-    const float mk = ceilf(seg_mask_max<W>(s, C0, L) * sl2);
-    float f = 1.f;                      // rescale of the earlier segments
-    if (C0 == 0) {
-        m = mk;
-    } else if (mk > m + kSlack) {
-        // 2^(m - mk) built from its exponent (m, mk are integers); below the
-        // normal range the old terms are negligible and drop to 0
-        const int e = (int)(m - mk);
-        f = e >= -126 ? __int_as_float((127 + e) << 23) : 0.f;
-        l *= f;
-        m = mk;
+    tmem_wait_ld();   // also completes a prefetch of the next segment
+    float mx = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < W; c += 16) {
+        uint32_t r[16];
+        tmem_ld16_nowait(tS + C0 + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            reg_fence(r[i]);
+            if (C0 + c + i < L)
+                mx = fmaxf(mx, __uint_as_float(r[i]));
+        }
     }
-    uint32_t pk[W / 2];
-    seg_exp<W>(s, pk, C0, L, sl2, m, l);
-    seg_store<W>(tS + C0 / 2, pk);
-    if (__any_sync(kFull, f != 1.f))    // after the store: few live registers
+    const float y = mx * sl2 - m;
+    const int k = y > 0.f ? (int)ceilf(y) : 0;
+    const float f = k <= 126 ? __int_as_float((127 - k) << 23) : 0.f;
+    m += (float)k;
+    l *= f;
+#pragma unroll 1
+    for (int c = 0; c < W; c += 16) {
+        uint32_t r[16], pk[8];
+        tmem_ld16_nowait(tS + C0 + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            reg_fence(r[2 * i]);
+            reg_fence(r[2 * i + 1]);
+            const float a = C0 + c + 2 * i < L ? ex2_approx(fmaf(__uint_as_float(r[2 * i]), sl2, -m)) : 0.f;
+            const float b = C0 + c + 2 * i + 1 < L ? ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), sl2, -m)) : 0.f;
+            l += a + b;
+            pk[i] = pack_bf16x2(a, b);
+        }
+        tmem_st8p(tS + (C0 + c) / 2, pk);
+        tmem_wait_st();
+    }
+    if (C0 > 0)
         rescale_p(tS, C0 / 2, f);
+}
+
+template <int NB, int SEG, int K>
+__device__ __forceinline__ void softmax_step(uint32_t tS, int L, float sl2, float &m, float &l, uint32_t (&cur)[SEG],
+                                             int trole, int tn)
+{
+    constexpr int C0 = K * SEG;
+    constexpr int W = NB - C0 < SEG ? NB - C0 : SEG;
+    constexpr int C1 = C0 + SEG;
+    if (K > 0) {
+        seg_issue<W>(tS + C0, cur);
+        tmem_wait_ld();
+        seg_fence<W>(cur);
+    }
+    if (C0 + W > L)   // warp-uniform
+        seg_mask<W>(cur, C0, L);
+    uint32_t pk[W / 2];
+    float ymax;
+    if (trole >= 0 && K < 4)
+        NLE_TRACE_AT(trole, tn, 5 + 2 * K);
+    const float ls = seg_exp<W>(cur, pk, sl2, m, ymax);
+    if (trole >= 0 && K < 4)
+        NLE_TRACE_AT(trole, tn, 6 + 2 * K);
+    if (__any_sync(kFull, !(ymax <= kYMax))) {
+        softmax_rare<W>(tS, C0, L, sl2, m, l);
+    } else {
+        l += ls;
+        seg_store<W>(tS + C0 / 2, pk);
+    }
+    if constexpr (C1 < NB) {
+        if (L > C1)
+            softmax_step<NB, SEG, K + 1>(tS, L, sl2, m, l, cur, trole, tn);
+    }
 }
 
 // Returns this lane's row sum; P (bf16) is left over the first NB/2 columns
 // of S.  Segments wholly at or past L are skipped (the MMAs stop at
 // ceil16(L) keys).
 template <int NB, int SEG>
-__device__ __forceinline__ float softmax_rows(uint32_t tS, int L, float sl2)
+__device__ __forceinline__ float softmax_rows(uint32_t tS, int L, float sl2, int trole = -1, int tn = 0)
 {
-    static_assert(SEG % 16 == 0 && NB <= 4 * SEG, "segments");
-    float m = 0.f, l = 0.f;
+    static_assert(SEG % 16 == 0 && SEG >= 16, "segments");
     constexpr int W0 = NB < SEG ? NB : SEG;
-    softmax_segment<0, W0>(tS, L, sl2, m, l);
-    if constexpr (NB > SEG) {
-        constexpr int W1 = NB - SEG < SEG ? NB - SEG : SEG;
-        if (L > SEG)
-            softmax_segment<SEG, W1>(tS, L, sl2, m, l);
-    }
-    if constexpr (NB > 2 * SEG) {
-        constexpr int W2 = NB - 2 * SEG < SEG ? NB - 2 * SEG : SEG;
-        if (L > 2 * SEG)
-            softmax_segment<2 * SEG, W2>(tS, L, sl2, m, l);
-    }
-    if constexpr (NB > 3 * SEG) {
-        constexpr int W3 = NB - 3 * SEG;
-        if (L > 3 * SEG)
-            softmax_segment<3 * SEG, W3>(tS, L, sl2, m, l);
-    }
+    uint32_t buf[SEG];
+    seg_issue<W0>(tS, buf);
+    tmem_wait_ld();
+    seg_fence<W0>(buf);
+    // first shift: max of the first 16 keys (keys >= L masked first)
+    if (W0 > L)
+        seg_mask<W0>(buf, 0, L);
+    float m = fmax3(fmax3(__uint_as_float(buf[0]), __uint_as_float(buf[1]), __uint_as_float(buf[2])),
+                    fmax3(__uint_as_float(buf[3]), __uint_as_float(buf[4]), __uint_as_float(buf[5])),
+                    fmax3(__uint_as_float(buf[6]), __uint_as_float(buf[7]), __uint_as_float(buf[8])));
+    m = fmax3(m, fmax3(__uint_as_float(buf[9]), __uint_as_float(buf[10]), __uint_as_float(buf[11])),
+              fmax3(fmax3(__uint_as_float(buf[12]), __uint_as_float(buf[13]), __uint_as_float(buf[14])),
+                    __uint_as_float(buf[15]), -INFINITY));
+    m *= sl2;
+    float l = 0.f;
+    softmax_step<NB, SEG, 0>(tS, L, sl2, m, l, buf, trole, tn);
+    if (trole >= 0)
+        NLE_TRACE_AT(trole, tn, 13);
     tmem_wait_st();
+    if (trole >= 0)
+        NLE_TRACE_AT(trole, tn, 14);
     return l;
 }
 
 template <int NB>
-__global__ void __launch_bounds__(Shape<NB>::threads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     block_attn_kernel(const __grid_constant__ CUtensorMap tm_q0, const __grid_constant__ CUtensorMap tm_q1,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                      const Params p)
+                      const __grid_constant__ CUtensorMap tm_o, const Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t qk_base = smem_u32(smem);
     const uint32_t v_off = p.sqk * p.qk_bytes;
     const uint32_t v_base = qk_base + v_off;
-    Bars *bars = reinterpret_cast<Bars *>(smem + v_off + kSV * p.v_bytes);
-    constexpr int kThreads = Shape<NB>::threads;
-    constexpr int kSoftmax0 = Shape<NB>::first_softmax_warp;
+    Bars *bars = reinterpret_cast<Bars *>(smem + p.stage_off + 8 * p.stage_bufs * 4096);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -294,20 +389,22 @@ __global__ void __launch_bounds__(Shape<NB>::threads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.sqk; ++s) {
             mbar_init(smem_u32(&bars->qk_full[s]), 1);
-            mbar_init(smem_u32(&bars->qk_empty[s]), 1);
+            mbar_init(smem_u32(&bars->qk_empty[s]), 2);
         }
         for (int s = 0; s < kSV; ++s) {
             mbar_init(smem_u32(&bars->v_full[s]), 1);
-            mbar_init(smem_u32(&bars->v_empty[s]), 1);
+            mbar_init(smem_u32(&bars->v_ready[s]), 1);
+            mbar_init(smem_u32(&bars->v_empty[s]), 2);
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(smem_u32(&bars->s_full[t]), 1);
-            mbar_init(smem_u32(&bars->p_full[t]), 4);
+            mbar_init(smem_u32(&bars->wg_p[t]), 4);
             mbar_init(smem_u32(&bars->o_full[t]), 1);
-            mbar_init(smem_u32(&bars->tmem_free[t]), 4);
+            mbar_init(smem_u32(&bars->wg_o[t]), 4);
+            mbar_init(smem_u32(&bars->mma_done[t]), 1);
         }
-        mbar_init(smem_u32(&bars->mma_done), 1);
         bars->abort_flag = 0;
+        bars->turn = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -319,6 +416,7 @@ __global__ void __launch_bounds__(Shape<NB>::threads, 1)
         tma_prefetch_desc(&tm_q1);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_o);
     }
     // V rows B..NB-1 (MMA padding) are zero for the whole launch.
     {
@@ -336,10 +434,11 @@ __global__ void __launch_bounds__(Shape<NB>::threads, 1)
     volatile int *abort_flag = &bars->abort_flag;
     const unsigned long long wait_ns = p.wait_ns;
     const int H = p.heads;
+    // work items of this CTA: item = blockIdx.x + n * gridDim.x = b * H + h
+    const int step_b = (int)(gridDim.x / H), step_h = (int)(gridDim.x % H);
+    const int first_b = (int)(blockIdx.x / H), first_h = (int)(blockIdx.x % H);
 
     if (warp < kSoftmax0) {
-        if constexpr (Shape<NB>::split)
-            regs_dec<kRegsLow>();
         if (warp == 0) {
             // ==================================================== producer
             PlanWalker w;
@@ -366,9 +465,7 @@ __global__ void __launch_bounds__(Shape<NB>::threads, 1)
                 return true;
             };
 
-            for (int item = blockIdx.x;; item += gridDim.x, ++n) {
-                const int b = item / H;
-                const int h = item - b * H;
+            for (int b = first_b, h = first_h;; ++n) {
                 int f0, L, seq;
                 if (!w.find(b, lane, f0, L, seq))
                     break;
@@ -398,6 +495,12 @@ __global__ void __launch_bounds__(Shape<NB>::threads, 1)
                 }
                 prev_h = h;
                 prev_f0 = f0;
+                b += step_b;
+                h += step_h;
+                if (h >= H) {
+                    h -= H;
+                    ++b;
+                }
             }
             if (ok && n > 0)
                 issue_v(n - 1, prev_h, prev_f0);
@@ -416,166 +519,294 @@ __global__ void __launch_bounds__(Shape<NB>::threads, 1)
                         wait_bar_drain(smem_u32(&bars->v_full[m % kSV]), (uint32_t)(m / kSV) & 1, wait_ns);
             }
             __syncwarp();
-        } else if (warp == 1) {
-            // ==================================================== MMA issuer
-            PlanWalker w;
-            w.init(p.cu, p.n_seq, p.total, p.B, lane);
-            const uint32_t id_pv = idesc_bf16_f32(128, 64, true);
-            uint32_t tile_uses[2] = {0, 0};
-            int n = 0;
-            for (int item = blockIdx.x;; item += gridDim.x, ++n) {
-                const int b = item / H;
-                int f0, L, seq;
-                if (!w.find(b, lane, f0, L, seq))
-                    break;
-                const int s = n % p.sqk;
-                if (!wait_bar(smem_u32(&bars->qk_full[s]), (uint32_t)(n / p.sqk) & 1, abort_flag, wait_ns,
-                              p.status))
-                    break;
-                tc_fence_after();
-                const int ntiles = L > kQTile ? 2 : 1;
-                const int nkeys = (L + 15) & ~15;   // MMA extent over keys
-                const uint32_t id_s = idesc_bf16_f32(128, nkeys, false);
-                const uint32_t qaddr = qk_base + s * p.qk_bytes;
-                const uint32_t kaddr = qaddr + p.q_bytes;
-                bool ok = true;
-                for (int t = 0; t < ntiles; ++t) {
-                    const uint32_t ut = tile_uses[t];
-                    if (ut > 0 &&
-                        !wait_bar(smem_u32(&bars->tmem_free[t]), (ut - 1) & 1, abort_flag, wait_ns, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (lane == 0) {
-                        // K steps of 16 elements = 32 bytes inside the
-                        // 128-byte swizzle atom: advance the start address
-                        const uint64_t da = smem_desc_sw128(qaddr + t * kQTile * kRowBytes, 16, 1024);
-                        const uint64_t db = smem_desc_sw128(kaddr, 16, 1024);
-#pragma unroll 1
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ss(tmem + t * kSlotCols, da + 2 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
-                        mma_commit(smem_u32(&bars->s_full[t]));
-                    }
-                    __syncwarp();
-                }
-                if (!ok)
-                    break;
-                if (lane == 0)
-                    mma_commit(smem_u32(&bars->qk_empty[s]));
-                __syncwarp();
-                const int sv = n % kSV;
-                if (!wait_bar(smem_u32(&bars->v_full[sv]), (uint32_t)(n / kSV) & 1, abort_flag, wait_ns,
-                              p.status))
-                    break;
-                // PV reads V rows 0..nkeys-1; rows L..nkeys-1 of a partial
-                // block hold frames of the next block (or utterance): zero
-                // them so nothing outside the block reaches PV (P is 0 there,
-                // but 0 * Inf would be NaN).  Rows B..NB-1 are always zero.
-                if (L < nkeys && L < p.B) {
-                    const int zend = nkeys < p.B ? nkeys : p.B;
-                    uint4 *vz = reinterpret_cast<uint4 *>(smem + v_off + sv * p.v_bytes + L * kRowBytes);
-                    for (int i = lane; i < (zend - L) * (kRowBytes / 16); i += 32)
-                        vz[i] = make_uint4(0, 0, 0, 0);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                }
-                tc_fence_after();
-                const uint32_t vaddr = v_base + sv * p.v_bytes;
-                for (int t = 0; t < ntiles; ++t) {
-                    const uint32_t ut = tile_uses[t];
-                    if (!wait_bar(smem_u32(&bars->p_full[t]), ut & 1, abort_flag, wait_ns, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t slot = tmem + t * kSlotCols;
-                        // N = 64 is one 128-byte swizzle atom along N, so the
-                        // N-direction atom stride (LBO) is never used; K steps
-                        // of 16 rows advance the start address by 2048 bytes.
-                        const uint64_t db = smem_desc_sw128(vaddr, 0, 1024);
-#pragma unroll 1
-                        for (int kk = 0; kk < nkeys / 16; ++kk)
-                            mma_ts(slot + kOCol, slot + kk * 8, db + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
-                                   kk > 0 ? 1u : 0u);
-                        mma_commit(smem_u32(&bars->o_full[t]));
-                    }
-                    __syncwarp();
-                    tile_uses[t] = ut + 1;
-                }
-                if (!ok)
-                    break;
-                if (lane == 0)
-                    mma_commit(smem_u32(&bars->v_empty[sv]));
-                __syncwarp();
-            }
-            // every MMA issued so far must finish before TMEM is released
-            if (lane == 0) {
-                mma_commit(smem_u32(&bars->mma_done));
-                wait_bar_drain(smem_u32(&bars->mma_done), 0, wait_ns);
-            }
-            __syncwarp();
         }
     } else {
-        if constexpr (Shape<NB>::split)
-            regs_inc<kRegsHigh>();
-        // ======================================================== softmax + epilogue
+        // ======================================================== tile warpgroups
+        // Warpgroup t drives TMEM slot t: its first warp's elected lane
+        // issues the slot's MMAs, all four warps run softmax and epilogue.
+        // The two warpgroups take turns on the softmax (the MUFU-bound
+        // phase): one runs it while the other waits on its MMAs or writes
+        // its output.  The turn order is block by block, slot 0 then slot 1.
         const int t = (warp - kSoftmax0) >> 2;     // tile slot
         const int qq = warp & 3;                   // TMEM lane quarter of this warp
-        const uint32_t tS = tmem + ((uint32_t)(qq * 32) << 16) + t * kSlotCols;
+        const bool leader = qq == 0;
+        const uint32_t slot = tmem + t * kSlotCols;
+        const uint32_t tS = slot + ((uint32_t)(qq * 32) << 16);
         const float sl2 = p.scale_log2;
+        const uint32_t id_pv = idesc_bf16_f32(128, 64, true);
+        // output staging of this warp: two buffers of 32 rows x 128 B,
+        // 128-byte swizzle
+        const uint32_t stage_u32 = smem_u32(smem + p.stage_off + (warp - kSoftmax0) * p.stage_bufs * 4096);
+        int stores = 0;
         PlanWalker w;
         w.init(p.cu, p.n_seq, p.total, p.B, lane);
-        uint32_t uses = 0;
-        for (int item = blockIdx.x;; item += gridDim.x) {
-            const int b = item / H;
-            const int h = item - b * H;
-            int f0, L, seq;
-            if (!w.find(b, lane, f0, L, seq))
+        volatile int *turn = &bars->turn;
+        int b = first_b, h = first_h;
+        int n = -1;          // index of the current block among this CTA's items
+        int c1 = 0;          // blocks seen so far that have rows in slot 1
+        uint32_t uses = 0;   // blocks this slot has computed
+        int f0 = 0, L = 0, hcur = 0, my_turn = 0, nkeys = 16;
+        bool ok = true;
+
+        // Advance to the next block with rows in this slot; on the way,
+        // slot 1 releases its share of the stages of blocks it skips.  The
+        // leader then issues the block's S MMA (after the slot's previous O
+        // has been read by all four warps).  False at the end of the work.
+        auto advance = [&]() -> bool {
+            for (;;) {
+                int sf0, sL, sseq;
+                if (!w.find(b, lane, sf0, sL, sseq))
+                    return false;
+                ++n;
+                const int hh = h;
+                b += step_b;
+                h += step_h;
+                if (h >= H) {
+                    h -= H;
+                    ++b;
+                }
+                const int c1_before = c1;
+                if (sL > kQTile)
+                    ++c1;
+                const int s = n % p.sqk, sv = n % kSV;
+                const uint32_t ph_qk = (uint32_t)(n / p.sqk) & 1, ph_v = (uint32_t)(n / kSV) & 1;
+                if (t == 1 && sL <= kQTile) {
+                    if (leader) {
+                        if (!wait_bar(smem_u32(&bars->qk_full[s]), ph_qk, abort_flag, wait_ns, p.status)) {
+                            ok = false;
+                            return false;
+                        }
+                        if (lane == 0)
+                            mbar_arrive(smem_u32(&bars->qk_empty[s]));
+                        if (!wait_bar(smem_u32(&bars->v_full[sv]), ph_v, abort_flag, wait_ns, p.status)) {
+                            ok = false;
+                            return false;
+                        }
+                        if (lane == 0)
+                            mbar_arrive(smem_u32(&bars->v_empty[sv]));
+                    }
+                    continue;
+                }
+                f0 = sf0;
+                L = sL;
+                hcur = hh;
+                nkeys = (L + 15) & ~15;   // MMA extent over keys
+                my_turn = n + c1_before + t;
+                if (leader) {
+                    if (lane == 0)
+                        NLE_TRACE_AT(1 + t, n, 0);
+                    if (!wait_bar(smem_u32(&bars->qk_full[s]), ph_qk, abort_flag, wait_ns, p.status)) {
+                        ok = false;
+                        return false;
+                    }
+                    if (lane == 0)
+                        NLE_TRACE_AT(1 + t, n, 1);
+                    if (uses > 0 &&
+                        !wait_bar(smem_u32(&bars->wg_o[t]), (uses - 1) & 1, abort_flag, wait_ns, p.status)) {
+                        ok = false;
+                        return false;
+                    }
+                    tc_fence_after();
+                    if (lane == 0)
+                        NLE_TRACE_AT(1 + t, n, 2);
+                    // K steps of 16 elements = 32 bytes inside the 128-byte
+                    // swizzle atom: advance the descriptor start address
+                    const uint32_t qaddr = qk_base + s * p.qk_bytes;
+                    const uint64_t da = smem_desc_sw128(qaddr + t * kQTile * kRowBytes, 16, 1024);
+                    const uint64_t db = smem_desc_sw128(qaddr + p.q_bytes, 16, 1024);
+                    const uint32_t id_s = idesc_bf16_f32(128, nkeys, false);
+                    if (elect_one()) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss(slot, da + 2 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
+                        mma_commit(smem_u32(&bars->s_full[t]));
+                        mma_commit(smem_u32(&bars->qk_empty[s]));
+                        NLE_TRACE_AT(1 + t, n, 3);
+                    }
+                    __syncwarp();
+                }
+                return true;
+            }
+        };
+
+        // Each pass: advance (the leader issues the next block's S MMA),
+        // write the previous block's output, then compute the current block.
+        uint32_t pk[32];
+        bool pending = false;          // pk holds rows of the previous block
+        int ef0 = 0, eL = 0, eh = 0, erow0 = 0;
+        for (;;) {
+            const bool have = advance();
+            if (!ok)
                 break;
-            if (t == 1 && L <= kQTile)
-                continue;
+            if (pending) {
+                if (erow0 + 32 <= eL) {
+                    // all 32 rows inside the block: stage (swizzled) and
+                    // store with one TMA box of 32 rows; two staging buffers
+                    // alternate
+                    const uint32_t buf = stage_u32 + (stores % p.stage_bufs) * 4096;
+                    if (stores >= p.stage_bufs) {
+                        // the store that used this buffer must have read it
+                        if (lane == 0) {
+                            if (p.stage_bufs == 2)
+                                bulk_wait_read1();
+                            else
+                                bulk_wait_read0();
+                        }
+                        __syncwarp();
+                    }
+                    // the row's base address is made opaque here so the
+                    // eight swizzled addresses are formed at the stores, not
+                    // hoisted out of the block loop
+                    uint32_t srow = buf + lane * 128;
+                    asm volatile("" : "+r"(srow));
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        st_shared_v4(srow + ((c ^ (lane & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                                     pk[4 * c + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tm_o, eh * 64, ef0 + erow0, buf);
+                        bulk_commit();
+                    }
+                    ++stores;
+                } else if (erow0 + lane < eL) {
+                    // rows past the block end are never written
+                    uint4 *dst =
+                        reinterpret_cast<uint4 *>(p.out + (size_t)(ef0 + erow0 + lane) * p.out_stride + eh * 64);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                }
+                pending = false;
+            }
+            if (!have)
+                break;
+            const int sv = n % kSV;
+            const uint32_t ph_v = (uint32_t)(n / kSV) & 1;
+            // ---------------------------------------------- softmax
             if (!wait_bar(smem_u32(&bars->s_full[t]), uses & 1, abort_flag, wait_ns, p.status))
                 break;
             tc_fence_after();
+            // wait for this slot's turn on the softmax (bounded)
+            if (kPingPong && *turn < my_turn) {
+                const uint64_t t0 = globaltimer_ns();
+                while (*turn < my_turn) {
+                    __nanosleep(32);
+                    if (*abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    if (globaltimer_ns() - t0 > wait_ns) {
+                        *abort_flag = 1;
+                        report(p.status, NLE_ERR_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!__all_sync(kFull, ok))
+                    break;
+            }
+            if (lane == 0 && qq == 0)
+                NLE_TRACE_AT(3 + t, n, 0);
             const int row0 = t * kQTile + qq * 32;   // first block row of this warp
             const bool active = row0 < L;
             float l = 1.f;
             if (active)
-                l = softmax_rows<NB, Shape<NB>::seg>(tS, L, sl2);
+                l = softmax_rows<NB, kSeg>(tS, L, sl2, (lane == 0 && qq == 0) ? 3 + t : -1, n);
+            if (lane == 0 && qq == 0)
+                NLE_TRACE_AT(3 + t, n, 1);
+            if (t == 0 && L < nkeys && L < p.B) {
+                // PV reads V rows 0..nkeys-1; rows L..nkeys-1 of a partial
+                // block hold frames of the next block (or utterance): zero
+                // them so nothing outside the block reaches PV (P is 0 there,
+                // but 0 * Inf would be NaN).  Rows B..NB-1 are always zero.
+                if (!wait_bar(smem_u32(&bars->v_full[sv]), ph_v, abort_flag, wait_ns, p.status))
+                    break;
+                const int zend = nkeys < p.B ? nkeys : p.B;
+                uint4 *vz = reinterpret_cast<uint4 *>(smem + v_off + sv * p.v_bytes + L * kRowBytes);
+                for (int i = qq * 32 + lane; i < (zend - L) * (kRowBytes / 16); i += 128)
+                    vz[i] = make_uint4(0, 0, 0, 0);
+                fence_proxy_async_smem();
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(smem_u32(&bars->p_full[t]));
+                mbar_arrive(smem_u32(&bars->wg_p[t]));
+            // ---------------------------------------------- O = P V
+            if (leader) {
+                if (!wait_bar(smem_u32(&bars->wg_p[t]), uses & 1, abort_flag, wait_ns, p.status))
+                    break;
+                if (lane == 0)
+                    *turn = my_turn + 1;   // the other slot may run its softmax
+                if (t == 0) {
+                    if (!wait_bar(smem_u32(&bars->v_full[sv]), ph_v, abort_flag, wait_ns, p.status))
+                        break;
+                    if (lane == 0)
+                        mbar_arrive(smem_u32(&bars->v_ready[sv]));   // tail rows zeroed
+                } else if (!wait_bar(smem_u32(&bars->v_ready[sv]), ph_v, abort_flag, wait_ns, p.status)) {
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0)
+                    NLE_TRACE_AT(1 + t, n, 5);
+                // N = 64 is one 128-byte swizzle atom along N, so the
+                // N-direction atom stride (LBO) is never used; K steps of 16
+                // rows advance the start address by 2048 bytes.
+                const uint64_t dv = smem_desc_sw128(v_base + sv * p.v_bytes, 0, 1024);
+                if (elect_one()) {
+                    for (int kk = 0; kk < nkeys / 16; ++kk)
+                        mma_ts(slot + kOCol, slot + kk * 8, dv + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
+                               kk > 0 ? 1u : 0u);
+                    mma_commit(smem_u32(&bars->o_full[t]));
+                    mma_commit(smem_u32(&bars->v_empty[sv]));
+                    NLE_TRACE_AT(1 + t, n, 6);
+                }
+                __syncwarp();
+            }
+            // ---------------------------------------------- read O
             if (!wait_bar(smem_u32(&bars->o_full[t]), uses & 1, abort_flag, wait_ns, p.status))
                 break;
             tc_fence_after();
-            uint32_t o[64];
+            if (lane == 0 && qq == 0)
+                NLE_TRACE_AT(3 + t, n, 2);
             if (active) {
-                tmem_ld32_nowait(tS + kOCol, &o[0]);
-                tmem_ld32_nowait(tS + kOCol + 32, &o[32]);
+                uint32_t o[64];
+#pragma unroll
+                for (int c = 0; c < 64; c += 16)
+                    tmem_ld16_nowait(tS + kOCol + c, &o[c]);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
                     reg_fence(o[i]);
+                const float inv = 1.f / l;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(smem_u32(&bars->tmem_free[t]));
-            const int r = row0 + lane;
-            if (active && r < L) {
-                const float inv = 1.f / l;
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (size_t)(f0 + r) * p.out_stride + h * 64);
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    dst[c] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
-                                        pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
-                                        pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
-                                        pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
-            }
+                mbar_arrive(smem_u32(&bars->wg_o[t]));
+            if (lane == 0 && qq == 0)
+                NLE_TRACE_AT(3 + t, n, 3);
             ++uses;
+            pending = active;
+            ef0 = f0;
+            eL = L;
+            eh = hcur;
+            erow0 = row0;
+        }
+        if (lane == 0 && stores > 0)
+            bulk_wait0();
+        __syncwarp();
+        // this slot's MMAs must finish before TMEM is released
+        if (leader) {
+            if (elect_one()) {
+                mma_commit(smem_u32(&bars->mma_done[t]));
+                wait_bar_drain(smem_u32(&bars->mma_done[t]), 0, wait_ns);
+            }
+            __syncwarp();
         }
     }
 
@@ -588,18 +819,16 @@ __global__ void __launch_bounds__(Shape<NB>::threads, 1)
     }
 }
 
-using BlockKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, Params);
+using BlockKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, Params);
 
 struct KernelInfo {
     BlockKernel fn;
-    int threads;
-    bool split;
 };
 
 template <int NB>
 KernelInfo kernel_nb()
 {
-    return {reinterpret_cast<BlockKernel>(block_attn_kernel<NB>), Shape<NB>::threads, Shape<NB>::split};
+    return {reinterpret_cast<BlockKernel>(block_attn_kernel<NB>)};
 }
 
 KernelInfo pick_kernel(int nb)
@@ -624,10 +853,8 @@ KernelInfo pick_kernel(int nb)
     }
 }
 
-// Per (NB/16, device): dynamic smem opted in so far, and whether the
-// register count of a split build was verified (1 ok, -1 refused).
+// Per (NB/16, device): dynamic smem opted in so far.
 int g_smem_set[17][64] = {};
-int g_regs_ok[17][64] = {};
 
 } // namespace
 
@@ -679,13 +906,21 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
     p.q_bytes = (uint32_t)((rows8 > kQTile ? rows8 : kQTile) * kRowBytes);
     p.qk_bytes = p.q_bytes + (uint32_t)(rows8 * kRowBytes);
     p.v_bytes = (uint32_t)(NB * kRowBytes);
-    const size_t fixed = (size_t)kSV * p.v_bytes + ((sizeof(Bars) + 127) / 128) * 128 + 1024;
+    // fixed part: V ring, output staging (per softmax warp 2 x 4 KB, or
+    // 4 KB when that would leave fewer than two QK stages), barriers,
+    // alignment slack
+    const size_t other = (size_t)kSV * p.v_bytes + ((sizeof(Bars) + 127) / 128) * 128 + 1024;
+    p.stage_bufs = 2;
+    if ((size_t)di.smem_optin < other + (size_t)8 * 8192 + 2 * (size_t)p.qk_bytes)
+        p.stage_bufs = 1;
+    const size_t fixed = other + (size_t)8 * 4096 * p.stage_bufs;
     int sqk = (int)(((size_t)di.smem_optin - fixed) / p.qk_bytes);
     if (sqk > kMaxQK)
         sqk = kMaxQK;
     if (sqk < 2)
         return NLE_ERR_UNSUPPORTED;
     p.sqk = sqk;
+    p.stage_off = (uint32_t)(sqk * p.qk_bytes + kSV * p.v_bytes);
     size_t smem = (size_t)sqk * p.qk_bytes + fixed;
     // One CTA per SM: it owns all 512 TMEM columns, so a second resident CTA
     // would only wait in tcgen05.alloc.  Ask for more than half the SM's
@@ -700,30 +935,17 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
     p.wait_ns = wait_limit_ns > 0 ? (unsigned long long)wait_limit_ns : 1000000000ull;
     p.flags = flags;
 
-    CUtensorMap tq0, tq1, tk, tv;
+    CUtensorMap tq0, tq1, tk, tv, to;
     const uint64_t cols = (uint64_t)dense, rows = (uint64_t)total_frames;
     if (!nle::encode_tmap_bf16_2d(&tq0, q, cols, rows, stride, 64, p.q0rows) ||
         !nle::encode_tmap_bf16_2d(&tq1, q, cols, rows, stride, 64, p.q1rows ? p.q1rows : p.q0rows) ||
         !nle::encode_tmap_bf16_2d(&tk, k, cols, rows, stride, 64, B) ||
-        !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, stride, 64, B))
+        !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, stride, 64, B) ||
+        !nle::encode_tmap_bf16_2d(&to, out, cols, rows, dense, 64, 32))
         return NLE_ERR_CUDA;
 
     const KernelInfo kern = pick_kernel(NB);
     const int slot = dev < 64 ? dev : 0;
-    if (kern.split) {
-        // setmaxnreg.inc waits until the block's launch allocation can cover
-        // the new split; it can only if every thread starts with exactly
-        // kRegsLaunch registers.
-        int &ok = g_regs_ok[NB / 16][slot];
-        if (ok == 0 || dev >= 64) {
-            cudaFuncAttributes fa;
-            if (cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(kern.fn)) != cudaSuccess)
-                return NLE_ERR_CUDA;
-            ok = fa.numRegs == kRegsLaunch ? 1 : -1;
-        }
-        if (ok != 1)
-            return NLE_ERR_UNSUPPORTED;
-    }
     int &set = g_smem_set[NB / 16][slot];
     if (dev >= 64 || set < (int)smem) {
         if (cudaFuncSetAttribute(reinterpret_cast<const void *>(kern.fn),
@@ -732,7 +954,7 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
         set = (int)smem;
     }
     const int grid = (int)(max_items < di.sm_count ? max_items : di.sm_count);
-    kern.fn<<<grid, kern.threads, smem, static_cast<cudaStream_t>(stream)>>>(tq0, tq1, tk, tv, p);
+    kern.fn<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tq0, tq1, tk, tv, to, p);
     return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
 }
 

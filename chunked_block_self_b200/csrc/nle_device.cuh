@@ -149,6 +149,11 @@ __device__ __forceinline__ uint64_t policy_evict_first()
     return p;
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 // Generic-proxy smem writes -> visible to the async proxy (TMA / tcgen05).
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
@@ -294,6 +299,42 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// One lane of the (converged) warp gets true.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t p;
+    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}" : "=r"(p));
+    return p != 0;
+}
+
+// 2-D tiled TMA store smem -> global (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const void *tmap, int32_t x, int32_t y, uint32_t src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until the smem sources of all committed bulk stores have been read.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Wait until the smem sources of all but the newest committed bulk store
+// group have been read.
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
+// Wait until all committed bulk stores have completed.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -318,6 +359,7 @@ struct PlanWalker {
     int incl;       // this lane's inclusive prefix of units within the group
     int start;      // cu[base + lane]
     int len;        // frames of utterance base + lane (0 if invalid/absent)
+    int units;      // units of utterance base + lane
     int group_units;
     int bad;        // warp-uniform: an invalid utterance was seen
 
@@ -337,6 +379,7 @@ struct PlanWalker {
         }
         start = a;
         len = b - a;
+        units = n;
         int x = n;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -379,7 +422,7 @@ struct PlanWalker {
         const int incl_s = __shfl_sync(kFull, incl, src);
         const int st = __shfl_sync(kFull, start, src);
         const int ln = __shfl_sync(kFull, len, src);
-        const int nb = (ln + unit - 1) / unit;
+        const int nb = __shfl_sync(kFull, units, src);
         const int j = rel - (incl_s - nb);
         frame0 = st + j * unit;
         L = min(unit, ln - j * unit);

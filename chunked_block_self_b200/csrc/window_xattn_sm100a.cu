@@ -8,16 +8,22 @@
 // an utterance may be partial) and owns query rows Qw*g .. Qw*g + Qw - 1;
 // each query row attends to the window's L frames, per head.
 //
-// The work is HBM-bound (about 2.5 flop per byte), so it runs on the CUDA
-// cores.  One persistent CTA per SM (8 warps) walks windows g = blockIdx.x,
-// blockIdx.x + gridDim.x, ...; the K rows, V rows and Q rows of a window are
-// each one contiguous range of memory ([frames][heads][64] layout), fetched
-// with a single bulk copy apiece into a ring of shared-memory stages.
-// Per window, each warp takes a pair of heads: in QK^T one lane per key
-// (half a warp per head, the 16-byte chunks of a key row visited in a
-// lane-rotated order so the shared-memory reads do not collide), softmax
-// by shuffles inside the half-warp, then PV with one lane per two output
-// dimensions and coalesced 4-byte bf16x2 stores.
+// The work is HBM-bound (about 2.5 flop per byte).  One persistent CTA per
+// SM walks windows g = blockIdx.x, blockIdx.x + gridDim.x, ...:
+//   warp 16     producer: per window one 128-byte-swizzled TMA box per head
+//               for K and for V (W rows of 64 bf16; no multicast) and one
+//               bulk copy for the window's contiguous query rows, into a
+//               ring of shared-memory stages.
+//   warps 0-15  one head each (heads h = warp, warp + 16, ...): the window's
+//               S = Q K^T (at most 16 queries x 16 keys) and O = P V are
+//               warp-level mma.sync m16n8k16 products (bf16 in, fp32
+//               accumulate) fed by ldmatrix from the swizzled tiles; softmax
+//               in fp32 with quad shuffles (keys >= L are 0 by index); P is
+//               reused from the accumulator registers as the A fragment of
+//               PV.  O is divided by the row sum, rounded to bf16 and written
+//               as coalesced 128-byte rows.
+// The tensor cores are used here only because the window's two products
+// are dense contractions that map onto one warp; the kernel's bound is HBM.
 #include <cmath>
 
 #include "nle.h"
@@ -28,13 +34,15 @@ namespace {
 
 using namespace nle;
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kMaxStages = 3;
-constexpr int kMaxQw = 8;
+constexpr int kComputeWarps = 16;
+constexpr int kThreads = (kComputeWarps + 1) * 32;
+constexpr int kMaxStages = 4;
+constexpr int kMaxQw = 16;
+constexpr int kTileBytes = 2048;   // 16 rows x 128 B, one head's keys (or values) per 16-key group
 
 struct WBars {
     uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];    // kComputeWarps arrivals
     int abort_flag;
 };
 
@@ -45,14 +53,15 @@ struct WParams {
     long long n_qrows;
     int heads;
     int W;        // window_frames
+    int box_rows; // rows of one K/V box: min(W, 16)
     int Qw;       // queries_per_window
-    const __nv_bfloat16 *q, *k, *v;
+    const __nv_bfloat16 *q;
     __nv_bfloat16 *out;
     int stages;
-    uint32_t kv_bytes;    // K (or V) region of a stage: W * heads * 128
-    uint32_t q_bytes;     // Q region: Qw * heads * 128
+    uint32_t kv_bytes;    // K (or V) region of a stage: heads * KT * 2048
+    uint32_t q_bytes;     // Q rows of a window: Qw * heads * 128
     uint32_t stage_bytes;
-    uint32_t qf_off;      // fp32 copy of the current window's queries
+    uint32_t ostage_off;  // per-warp output staging (Qw x 128 B each)
     uint32_t bars_off;
     float scale_log2;
     int32_t *status;
@@ -60,230 +69,285 @@ struct WParams {
     int flags;
 };
 
-__device__ __forceinline__ void unpack8(const uint4 &x, float (&f)[8])
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
 {
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr)
+                 : "memory");
 }
 
-// KPL = lanes per head group: 16 (two heads per warp, W <= 16) or 32.
-// QW = queries per window.
-template <int KPL, int QW>
-__global__ void __launch_bounds__(kThreads, 1) window_xattn_kernel(const WParams p)
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr)
+                 : "memory");
+}
+
+// D = A * B + D, m16n8k16, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of (row, 16-byte chunk) in a 128-byte-swizzled tile whose
+// base is 1024-byte aligned.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+// KT = number of 16-key groups (window_frames <= 16 * KT).
+template <int KT>
+__global__ void __launch_bounds__(kThreads, 1)
+    window_xattn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const WParams p)
 {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     WBars *bars = reinterpret_cast<WBars *>(smem + p.bars_off);
-    float *qf = reinterpret_cast<float *>(smem + p.qf_off);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int H = p.heads;
     const long long row_elems = (long long)H * 64;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < p.stages; ++s)
+        for (int s = 0; s < p.stages; ++s) {
             mbar_init(smem_u32(&bars->full[s]), 1);
+            mbar_init(smem_u32(&bars->empty[s]), kComputeWarps);
+        }
         bars->abort_flag = 0;
         fence_mbar_init();
     }
+    if (threadIdx.x == 32) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    // With one 16-key group (W <= 16), value rows W..15 of every head tile
+    // are MMA padding: never loaded, always zero (P is 0 there, and 0 * NaN
+    // would not be).  With two groups the boxes are 16 rows and rows past W
+    // are zeroed per window below.
+    if (KT == 1) {
+        const int pad_rows = 16 - p.W;
+        const int per_stage = H * KT * pad_rows * 8;   // 16-byte chunks
+        for (int i = threadIdx.x; i < p.stages * per_stage; i += kThreads) {
+            const int s = i / per_stage, r = i - s * per_stage;
+            const int tile = r / (pad_rows * 8), c = r - tile * pad_rows * 8;
+            uint8_t *vt = smem + s * p.stage_bytes + p.kv_bytes + tile * kTileBytes;
+            reinterpret_cast<uint4 *>(vt + (16 - pad_rows) * 128)[c] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+    }
     __syncthreads();
     volatile int *abort_flag = &bars->abort_flag;
+    const unsigned long long wait_ns = p.wait_ns;
 
-    // ------------------------------------------------ producer (warp 0)
-    PlanWalker pw;
-    uint64_t pol = 0;
-    long long issued = 0;      // windows issued so far (local index)
-    bool prod_done = false;
-    if (warp == 0) {
-        pw.init(p.cu, p.n_seq, p.total, p.W, lane);
-        pol = policy_evict_first();
-    }
-    auto issue = [&](long long n) {
-        const long long g = blockIdx.x + n * (long long)gridDim.x;
-        int f0, L, seq;
-        if (!pw.find(g, lane, f0, L, seq)) {
-            prod_done = true;
-            return;
-        }
-        if (lane == 0 && !((p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) && n == 0)) {
-            const int s = (int)(n % p.stages);
-            const uint32_t bar = smem_u32(&bars->full[s]);
-            const uint32_t dst = smem_u32(smem + s * p.stage_bytes);
-            if ((long long)p.Qw * (g + 1) > p.n_qrows) {
-                mbar_arrive(bar);   // no data: consumers skip this window
-            } else {
-                const uint32_t kvb = (uint32_t)L * H * 128u;
-                mbar_arrive_expect_tx(bar, 2 * kvb + p.q_bytes);
-                bulk_load(dst, p.k + (long long)f0 * row_elems, kvb, bar, pol);
-                bulk_load(dst + p.kv_bytes, p.v + (long long)f0 * row_elems, kvb, bar, pol);
-                bulk_load(dst + 2 * p.kv_bytes, p.q + (long long)p.Qw * g * row_elems, p.q_bytes, bar, pol);
+    if (warp == kComputeWarps) {
+        // ======================================================== producer
+        PlanWalker w;
+        w.init(p.cu, p.n_seq, p.total, p.W, lane);
+        const uint64_t pol = policy_evict_first();
+        int n = 0;
+        for (;; ++n) {
+            const long long g = blockIdx.x + (long long)n * gridDim.x;
+            int f0, L, seq;
+            if (!w.find(g, lane, f0, L, seq))
+                break;
+            const int s = n % p.stages;
+            const uint32_t u = (uint32_t)(n / p.stages);
+            if (u > 0 && !wait_bar(smem_u32(&bars->empty[s]), (u - 1) & 1, abort_flag, wait_ns, p.status))
+                break;
+            if (lane == 0 && !((p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) && n == 0)) {
+                const uint32_t bar = smem_u32(&bars->full[s]);
+                const uint32_t st = smem_u32(smem + s * p.stage_bytes);
+                if ((long long)p.Qw * (g + 1) > p.n_qrows) {
+                    mbar_arrive(bar);   // no query rows: consumers skip this window
+                } else {
+                    mbar_arrive_expect_tx(bar, 2u * H * KT * (uint32_t)p.box_rows * 128u + p.q_bytes);
+                    for (int h = 0; h < H; ++h) {
+                        for (int kt = 0; kt < KT; ++kt) {
+                            // one box of min(W, 16) rows per 16-key group
+                            tma_load_2d(st + (h * KT + kt) * kTileBytes, &tm_k, h * 64, f0 + 16 * kt, bar, pol);
+                            tma_load_2d(st + p.kv_bytes + (h * KT + kt) * kTileBytes, &tm_v, h * 64, f0 + 16 * kt,
+                                        bar, pol);
+                        }
+                    }
+                    bulk_load(st + 2 * p.kv_bytes, p.q + (long long)p.Qw * g * row_elems, p.q_bytes, bar, pol);
+                }
             }
+            __syncwarp();
+        }
+        if (w.bad && lane == 0)
+            report(p.status, NLE_ERR_INVALID_ARG);
+        // drain: the last copy into each stage must land before exit
+        if (lane == 0) {
+            const bool skipped0 = (p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) != 0;
+            for (int m = n - p.stages; m < n; ++m)
+                if (m >= 0 && !(skipped0 && m == 0))
+                    wait_bar_drain(smem_u32(&bars->full[m % p.stages]), (uint32_t)(m / p.stages) & 1, wait_ns);
         }
         __syncwarp();
-        issued = n + 1;
-    };
-    if (warp == 0)
-        for (long long n = 0; n < p.stages - 1 && !prod_done; ++n)
-            issue(n);
-
-    // ------------------------------------------------ consumers (all warps)
-    PlanWalker cw;
-    cw.init(p.cu, p.n_seq, p.total, p.W, lane);
-    const float sl2 = p.scale_log2;
-    long long n = 0;
-    for (;; ++n) {
-        if (warp == 0 && !prod_done)
-            issue(n + p.stages - 1);
-        const long long g = blockIdx.x + n * (long long)gridDim.x;
-        int f0, L, seq;
-        if (!cw.find(g, lane, f0, L, seq))
-            break;
-        const int s = (int)(n % p.stages);
-        const bool ok = wait_bar(smem_u32(&bars->full[s]), (uint32_t)(n / p.stages) & 1, abort_flag, p.wait_ns,
-                                 p.status);
-        if (__syncthreads_or(!ok))
-            break;
-        const bool q_ok = (long long)p.Qw * (g + 1) <= p.n_qrows;
-        const uint8_t *st = smem + s * p.stage_bytes;
-        if (q_ok) {
-            // queries of this window -> fp32 (read many times below)
-            const uint4 *qs = reinterpret_cast<const uint4 *>(st + 2 * p.kv_bytes);
-            const int chunks = p.Qw * H * 8;
-            for (int i = threadIdx.x; i < chunks; i += kThreads) {
-                float f[8];
-                unpack8(qs[i], f);
-                float4 *d = reinterpret_cast<float4 *>(qf + i * 8);
-                d[0] = make_float4(f[0], f[1], f[2], f[3]);
-                d[1] = make_float4(f[4], f[5], f[6], f[7]);
+    } else {
+        // ======================================================== heads
+        PlanWalker w;
+        w.init(p.cu, p.n_seq, p.total, p.W, lane);
+        const float sl2 = p.scale_log2;
+        const int gq = lane >> 2;       // fragment row group (query)
+        const int tq = lane & 3;        // thread in group
+        uint8_t *ost = smem + p.ostage_off + warp * p.Qw * 128;
+        for (int n = 0;; ++n) {
+            const long long g = blockIdx.x + (long long)n * gridDim.x;
+            int f0, L, seq;
+            if (!w.find(g, lane, f0, L, seq))
+                break;
+            const int s = n % p.stages;
+            if (!wait_bar(smem_u32(&bars->full[s]), (uint32_t)(n / p.stages) & 1, abort_flag, wait_ns, p.status))
+                break;
+            const bool q_ok = (long long)p.Qw * (g + 1) <= p.n_qrows;
+            uint8_t *st = smem + s * p.stage_bytes;
+            const uint32_t kbase = smem_u32(st), vbase = kbase + p.kv_bytes, qbase = kbase + 2 * p.kv_bytes;
+            for (int h = warp; q_ok && h < H; h += kComputeWarps) {
+                // ---- S = Q K^T: A = queries (rows >= Qw repeat query rows),
+                // B = keys of this head (n-tiles of 8 keys)
+                float sacc[2 * KT][4];
+#pragma unroll
+                for (int j = 0; j < 2 * KT; ++j)
+                    sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+                const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;   // row this lane addresses in ldmatrix
+                const int aq = arow % p.Qw;
+                const uint32_t qrow = qbase + (uint32_t)((aq * H + h) * 128);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t a[4];
+                    ldsm_x4(qrow + (2 * ks + (lane >> 4)) * 16, a[0], a[1], a[2], a[3]);
+#pragma unroll
+                    for (int kt = 0; kt < KT; ++kt) {
+                        // matrices: (keys 0-7, dims lo), (keys 0-7, dims hi),
+                        // (keys 8-15, dims lo), (keys 8-15, dims hi)
+                        const int krow = (lane & 7) + (lane >> 4) * 8;
+                        const int kchunk = 2 * ks + ((lane >> 3) & 1);
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(kbase + (h * KT + kt) * kTileBytes + swz(krow, kchunk), b0, b1, b2, b3);
+                        mma_16816(sacc[2 * kt], a, b0, b1);
+                        mma_16816(sacc[2 * kt + 1], a, b2, b3);
+                    }
+                }
+                // ---- softmax over the keys of each query row (quad = row)
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 2 * KT; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int key = 8 * j + 2 * tq + e;
+                        if (key >= L) {
+                            sacc[j][e] = -INFINITY;
+                            sacc[j][2 + e] = -INFINITY;
+                        }
+                        mx0 = fmaxf(mx0, sacc[j][e]);
+                        mx1 = fmaxf(mx1, sacc[j][2 + e]);
+                    }
+                }
+                mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
+                const float m0 = mx0 * sl2, m1 = mx1 * sl2;
+                float l0 = 0.f, l1 = 0.f;
+                uint32_t pa[KT][4];   // P as the A fragment of PV, per 16-key group
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+                    float pv[2][4];
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int j = 2 * kt + jj;
+                        pv[jj][0] = ex2_approx(fmaf(sacc[j][0], sl2, -m0));
+                        pv[jj][1] = ex2_approx(fmaf(sacc[j][1], sl2, -m0));
+                        pv[jj][2] = ex2_approx(fmaf(sacc[j][2], sl2, -m1));
+                        pv[jj][3] = ex2_approx(fmaf(sacc[j][3], sl2, -m1));
+                        l0 += pv[jj][0] + pv[jj][1];
+                        l1 += pv[jj][2] + pv[jj][3];
+                    }
+                    pa[kt][0] = pack_bf16x2(pv[0][0], pv[0][1]);   // row g,   keys 2t..
+                    pa[kt][1] = pack_bf16x2(pv[0][2], pv[0][3]);   // row g+8, keys 2t..
+                    pa[kt][2] = pack_bf16x2(pv[1][0], pv[1][1]);   // row g,   keys 8+2t..
+                    pa[kt][3] = pack_bf16x2(pv[1][2], pv[1][3]);   // row g+8, keys 8+2t..
+                }
+                l0 += __shfl_xor_sync(kFull, l0, 1);
+                l0 += __shfl_xor_sync(kFull, l0, 2);
+                l1 += __shfl_xor_sync(kFull, l1, 1);
+                l1 += __shfl_xor_sync(kFull, l1, 2);
+                // ---- a partial window: value rows L..W-1 hold frames of the
+                // next window (or utterance); zero them so nothing outside
+                // the window reaches PV
+                const int zr_end = KT == 1 ? p.W : 16 * KT;   // rows a TMA box may have filled
+                if (L < zr_end) {
+                    for (int i = lane; i < (zr_end - L) * 8; i += 32) {
+                        const int r = L + i / 8, c = i % 8;
+                        const int kt = r >> 4;
+                        *reinterpret_cast<uint4 *>(st + p.kv_bytes + (h * KT + kt) * kTileBytes + swz(r & 15, c)) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    __syncwarp();
+                }
+                // ---- O = P V: B = values via transposing ldmatrix
+                float oacc[8][4];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+#pragma unroll
+                for (int kt = 0; kt < KT; ++kt) {
+#pragma unroll
+                    for (int jp = 0; jp < 4; ++jp) {
+                        // matrices: (keys 0-7, dims 16jp..), (keys 8-15, dims 16jp..),
+                        // (keys 0-7, dims 16jp+8..), (keys 8-15, dims 16jp+8..)
+                        const int vrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+                        const int vchunk = 2 * jp + (lane >> 4);
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_t(vbase + (h * KT + kt) * kTileBytes + swz(vrow, vchunk), b0, b1, b2, b3);
+                        mma_16816(oacc[2 * jp], pa[kt], b0, b1);
+                        mma_16816(oacc[2 * jp + 1], pa[kt], b2, b3);
+                    }
+                }
+                // ---- normalise, stage the Qw rows of this head, write them
+                // as coalesced 128-byte rows
+                const float inv0 = 1.f / l0;
+                if (gq < p.Qw) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint32_t *>(ost + gq * 128 + j * 16 + tq * 4) =
+                            pack_bf16x2(oacc[j][0] * inv0, oacc[j][1] * inv0);
+                }
+                if (gq + 8 < p.Qw) {
+                    const float inv1 = 1.f / l1;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint32_t *>(ost + (gq + 8) * 128 + j * 16 + tq * 4) =
+                            pack_bf16x2(oacc[j][2] * inv1, oacc[j][3] * inv1);
+                }
+                __syncwarp();
+                for (int r = 0; r < p.Qw; ++r) {
+                    const uint32_t v = *reinterpret_cast<const uint32_t *>(ost + r * 128 + lane * 4);
+                    *reinterpret_cast<uint32_t *>(p.out + ((long long)p.Qw * g + r) * row_elems + h * 64 + 2 * lane) = v;
+                }
+                __syncwarp();
             }
+            if (!q_ok && warp == 0 && lane == 0)
+                report(p.status, NLE_ERR_INVALID_ARG);
+            // generic writes (zeroed rows) before the stage is refilled by TMA
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bars->empty[s]));
         }
-        __syncthreads();
-        if (q_ok) {
-            const uint8_t *ks = st;
-            const uint8_t *vs = st + p.kv_bytes;
-            constexpr int HPG = 32 / KPL;          // heads per warp pass
-            const int sub = lane / KPL;
-            const int j = lane % KPL;               // key handled in QK^T
-            for (int pair = warp; pair * HPG < H; pair += kWarps) {
-                const int head = pair * HPG + sub;
-                const bool kv_ok = head < H && j < L;
-                float sc[QW];
-#pragma unroll
-                for (int r = 0; r < QW; ++r)
-                    sc[r] = 0.f;
-                if (kv_ok) {
-                    const uint4 *krow = reinterpret_cast<const uint4 *>(ks + ((size_t)j * H + head) * 128);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const int cc = (c + j) & 7;
-                        float kf[8];
-                        unpack8(krow[cc], kf);
-#pragma unroll
-                        for (int r = 0; r < QW; ++r) {
-                            {
-                                const float4 *qp = reinterpret_cast<const float4 *>(qf + ((size_t)(r * H + head) * 64 + cc * 8));
-                                const float4 a = qp[0], b = qp[1];
-                                sc[r] = fmaf(a.x, kf[0], sc[r]);
-                                sc[r] = fmaf(a.y, kf[1], sc[r]);
-                                sc[r] = fmaf(a.z, kf[2], sc[r]);
-                                sc[r] = fmaf(a.w, kf[3], sc[r]);
-                                sc[r] = fmaf(b.x, kf[4], sc[r]);
-                                sc[r] = fmaf(b.y, kf[5], sc[r]);
-                                sc[r] = fmaf(b.z, kf[6], sc[r]);
-                                sc[r] = fmaf(b.w, kf[7], sc[r]);
-                            }
-                        }
-                    }
-                }
-                // softmax over the keys of this head group (fp32, exp2)
-#pragma unroll
-                for (int r = 0; r < QW; ++r) {
-                    {
-                        const float x = kv_ok ? sc[r] * sl2 : -INFINITY;
-                        float m = x;
-#pragma unroll
-                        for (int o = KPL / 2; o >= 1; o >>= 1)
-                            m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-                        const float e = kv_ok ? ex2_approx(x - m) : 0.f;
-                        float sum = e;
-#pragma unroll
-                        for (int o = KPL / 2; o >= 1; o >>= 1)
-                            sum += __shfl_xor_sync(kFull, sum, o);
-                        sc[r] = kv_ok ? e / sum : 0.f;
-                    }
-                }
-                // PV: lane owns output dims 2*lane, 2*lane+1
-#pragma unroll
-                for (int hs = 0; hs < HPG; ++hs) {
-                    const int hh = pair * HPG + hs;
-                    if (hh >= H)
-                        break;
-                    float o[QW][2];
-#pragma unroll
-                    for (int r = 0; r < QW; ++r)
-                        o[r][0] = o[r][1] = 0.f;
-                    for (int jj = 0; jj < L; ++jj) {
-                        const uint32_t vv =
-                            *reinterpret_cast<const uint32_t *>(vs + ((size_t)jj * H + hh) * 128 + lane * 4);
-                        const float v0 = __uint_as_float(vv << 16), v1 = __uint_as_float(vv & 0xffff0000u);
-#pragma unroll
-                        for (int r = 0; r < QW; ++r) {
-                            {
-                                const float pr = __shfl_sync(kFull, sc[r], hs * KPL + jj);
-                                o[r][0] = fmaf(pr, v0, o[r][0]);
-                                o[r][1] = fmaf(pr, v1, o[r][1]);
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int r = 0; r < QW; ++r) {
-                        {
-                            __nv_bfloat16 *dst = p.out + ((long long)p.Qw * g + r) * row_elems + hh * 64 + 2 * lane;
-                            *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(o[r][0], o[r][1]);
-                        }
-                    }
-                }
-            }
-        } else if (threadIdx.x == 0) {
+        if (w.bad && warp == 0 && lane == 0)
             report(p.status, NLE_ERR_INVALID_ARG);
-        }
-        __syncthreads();
-    }
-    if (warp == 0) {
-        if (cw.bad && lane == 0)
-            report(p.status, NLE_ERR_INVALID_ARG);
-        // drain copies issued but not consumed (only after an abort)
-        if (lane == 0)
-            for (long long m = n; m < issued; ++m)
-                if (!((p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) && m == 0))
-                    wait_bar_drain(smem_u32(&bars->full[m % p.stages]), (uint32_t)(m / p.stages) & 1, p.wait_ns);
-        __syncwarp();
     }
     __syncthreads();
 }
 
-using WKernel = void (*)(const WParams);
-
-template <int KPL>
-WKernel pick_qw(int qw)
-{
-    switch (qw) {
-    case 1: return window_xattn_kernel<KPL, 1>;
-    case 2: return window_xattn_kernel<KPL, 2>;
-    case 3: return window_xattn_kernel<KPL, 3>;
-    case 4: return window_xattn_kernel<KPL, 4>;
-    case 5: return window_xattn_kernel<KPL, 5>;
-    case 6: return window_xattn_kernel<KPL, 6>;
-    case 7: return window_xattn_kernel<KPL, 7>;
-    default: return window_xattn_kernel<KPL, 8>;
-    }
-}
-
-int g_smem_set[2][kMaxQw + 1][64] = {};
+using WKernel = void (*)(CUtensorMap, CUtensorMap, WParams);
+int g_smem_set[3][64] = {};
 
 } // namespace
 
@@ -313,6 +377,7 @@ extern "C" int nle_window_xattn_fwd_ex(const void *q, const void *k, const void 
     if (di.cc_major != 10)
         return NLE_ERR_UNSUPPORTED;
 
+    const int KT = window_frames <= 16 ? 1 : 2;
     WParams p{};
     p.cu = cu_seqlens_kv;
     p.n_seq = n_seq;
@@ -320,44 +385,49 @@ extern "C" int nle_window_xattn_fwd_ex(const void *q, const void *k, const void 
     p.n_qrows = n_query_rows;
     p.heads = heads;
     p.W = window_frames;
+    p.box_rows = window_frames < 16 ? window_frames : 16;
     p.Qw = queries_per_window;
     p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.k = static_cast<const __nv_bfloat16 *>(k);
-    p.v = static_cast<const __nv_bfloat16 *>(v);
     p.out = static_cast<__nv_bfloat16 *>(out);
-    p.kv_bytes = (uint32_t)window_frames * heads * 128u;
+    p.kv_bytes = (uint32_t)heads * KT * kTileBytes;
     p.q_bytes = (uint32_t)queries_per_window * heads * 128u;
-    p.stage_bytes = (2 * p.kv_bytes + p.q_bytes + 127) / 128 * 128;
-    const size_t qf_bytes = (size_t)queries_per_window * heads * 64 * 4;
-    const size_t fixed = qf_bytes + ((sizeof(WBars) + 127) / 128) * 128 + 128;
-    if ((size_t)heads * 128u * (2 * window_frames + queries_per_window) > (size_t)di.smem_optin)
+    p.stage_bytes = (2 * p.kv_bytes + p.q_bytes + 1023) / 1024 * 1024;
+    const size_t ostage = (size_t)kComputeWarps * queries_per_window * 128;
+    const size_t fixed = ostage + ((sizeof(WBars) + 127) / 128) * 128 + 1024;
+    if ((size_t)di.smem_optin < fixed + 2 * (size_t)p.stage_bytes)
         return NLE_ERR_UNSUPPORTED;
     int stages = (int)(((size_t)di.smem_optin - fixed) / p.stage_bytes);
     if (stages > kMaxStages)
         stages = kMaxStages;
-    if (stages < 2)
-        return NLE_ERR_UNSUPPORTED;
     p.stages = stages;
-    p.qf_off = stages * p.stage_bytes;
-    p.bars_off = p.qf_off + (uint32_t)((qf_bytes + 127) / 128 * 128);
-    const size_t smem = (size_t)p.bars_off + ((sizeof(WBars) + 127) / 128) * 128 + 128;
+    p.ostage_off = stages * p.stage_bytes;
+    p.bars_off = p.ostage_off + (uint32_t)ostage;
+    const size_t smem = (size_t)p.bars_off + ((sizeof(WBars) + 127) / 128) * 128 + 1024;
     const double scale = softmax_scale > 0.f ? (double)softmax_scale : 1.0 / std::sqrt((double)d_head);
     p.scale_log2 = (float)(scale * 1.4426950408889634);
     p.status = dev_status;
     p.wait_ns = wait_limit_ns > 0 ? (unsigned long long)wait_limit_ns : 1000000000ull;
     p.flags = flags;
 
-    const bool half = window_frames <= 16;
-    WKernel kern = half ? pick_qw<16>(queries_per_window) : pick_qw<32>(queries_per_window);
-    int &set = g_smem_set[half][queries_per_window][dev < 64 ? dev : 0];
+    // K/V tensor maps: [total_frames][heads*64] bf16, boxes of 64 x min(16, W)
+    // rows (one 16-key group), 128-byte swizzle, zero fill past the end
+    CUtensorMap tk, tv;
+    const uint64_t cols = (uint64_t)heads * 64, rows = (uint64_t)total_frames;
+    if (!nle::encode_tmap_bf16_2d(&tk, k, cols, rows, cols, 64, (uint32_t)p.box_rows) ||
+        !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, cols, 64, (uint32_t)p.box_rows))
+        return NLE_ERR_CUDA;
+
+    WKernel kern = KT == 1 ? window_xattn_kernel<1> : window_xattn_kernel<2>;
+    int &set = g_smem_set[KT][dev < 64 ? dev : 0];
     if (dev >= 64 || set < (int)smem) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        if (cudaFuncSetAttribute(reinterpret_cast<const void *>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
             return NLE_ERR_CUDA;
         set = (int)smem;
     }
     const long long max_windows = (long long)n_seq + total_frames / window_frames;
     const int grid = (int)(max_windows < di.sm_count ? max_windows : di.sm_count);
-    kern<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
+    kern<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
 }
 

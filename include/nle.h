@@ -127,7 +127,7 @@ int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v,
  * k, v            device bf16 [total_frames][heads][64]
  * cu_seqlens_kv   device int32 [n_seq + 1] over the key/value frames
  * window_frames   1..32 (15 on the pages)
- * queries_per_window 1..8 (3 on the pages)
+ * queries_per_window 1..16 (3 on the pages)
  */
 int nle_window_xattn_fwd(const void *q, const void *k, const void *v,
                          void *out, const int32_t *cu_seqlens_kv, int n_seq,

@@ -71,7 +71,7 @@ def test_window_host_validation():
     assert f(*bad) == nle.NLE_ERR_UNSUPPORTED
     bad = list(base); bad[10] = 33
     assert f(*bad) == nle.NLE_ERR_UNSUPPORTED
-    bad = list(base); bad[11] = 9
+    bad = list(base); bad[11] = 17
     assert f(*bad) == nle.NLE_ERR_UNSUPPORTED
     bad = list(base); bad[11] = 0
     assert f(*bad) == nle.NLE_ERR_INVALID_ARG

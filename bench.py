@@ -42,19 +42,34 @@ METRIC = "block-attn TFLOP/s & encoder frames/s on 1 B200; % of dense BF16 peak"
 CFG = 4
 B, W, QW, D = 200, 15, 3, 64
 
-# ncu DRAM traffic of the block-attention kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum), captured on the source whose hash is given; per
-# unit of algorithmic bytes, so it scales to any launch.  Reported only while
-# the kernel source is unchanged.
-NCU_TRAFFIC = {"source_sha256": None, "traffic_over_algorithmic": None}
+# ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of each
+# kernel on the batch-128 workload, per unit of algorithmic bytes so that it
+# scales to any launch; valid only for the kernel source whose hash is given
+# (reported as null once the source changes).  Read below 1.0: part of the
+# output is still dirty in the 126 MB L2 when the launch ends.
+NCU_TRAFFIC = {
+    "block_attn": {"files": ("block_attn_sm100a.cu", "nle_device.cuh"),
+                   "source_sha256": "bd01f1db9296212ab371ceec86f286f8efc0449234c4bb6c5b85d2f1b6f8fefd",
+                   "traffic_over_algorithmic": (380182784 + 65091328) / 482533376},
+    "window_xattn": {"files": ("window_xattn_sm100a.cu", "nle_device.cuh"),
+                     "source_sha256": "378de2cb009b4a847389da8cd00033afaddbd67b022430687b545329552ccc35",
+                     "traffic_over_algorithmic": (265871360 + 7391232) / 290320384},
+}
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(kernel: str = "block_attn") -> str:
     h = hashlib.sha256()
-    for f in ("block_attn_sm100a.cu", "nle_device.cuh"):
+    for f in NCU_TRAFFIC[kernel]["files"]:
         with open(os.path.join(ROOT, "chunked_block_self_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
+
+
+def ncu_traffic(kernel: str, algorithmic_bytes: int):
+    e = NCU_TRAFFIC[kernel]
+    if e["source_sha256"] != kernel_source_sha(kernel):
+        return None
+    return e["traffic_over_algorithmic"] * algorithmic_bytes
 
 
 def measured_peaks():
@@ -178,17 +193,19 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ------------------------------------------------------------------ CPU oracle timing
 def oracle_sample(lengths, q, k, v, cu, qw, kw, vw, heads, budget_s: float):
-    """Time the fp64 oracle on whole utterances of the workload, in order,
-    until `budget_s` seconds have passed.  Returns (flops, frames, seconds,
-    utterances, threads)."""
+    """Time the fp64 oracle on whole utterances of the workload, in order
+    (wrapping around to the first utterance after the last), until `budget_s`
+    seconds have passed.  Returns (flops, frames, seconds, utterances,
+    threads)."""
     import oracle
+    starts = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    qstarts = np.concatenate([[0], np.cumsum([QW * -(-int(t) // W) for t in lengths])]).astype(np.int64)
     flops = frames = 0
     n_utt = 0
     t0 = time.perf_counter()
-    qrow = 0
-    a = 0
-    while n_utt < len(lengths) and time.perf_counter() - t0 < budget_s:
-        t = int(lengths[n_utt])
+    while n_utt == 0 or time.perf_counter() - t0 < budget_s:
+        i = n_utt % len(lengths)
+        t, a, qrow = int(lengths[i]), int(starts[i]), int(qstarts[i])
         local = np.array([0, t], np.int32)
         oracle.block_attn(q[a:a + t], k[a:a + t], v[a:a + t], local, block_frames=B, n_threads=0)
         nw = -(-t // W)
@@ -197,8 +214,6 @@ def oracle_sample(lengths, q, k, v, cu, qw, kw, vw, heads, budget_s: float):
         f2, _, _ = window_work([t], heads)
         flops += f1 + f2
         frames += t
-        a += t
-        qrow += QW * nw
         n_utt += 1
     return flops, frames, time.perf_counter() - t0, n_utt, oracle.threads_used(0)
 
@@ -365,14 +380,13 @@ def run_nle(args, rank, world, local):
                                               heads, args.cpu_seconds)
         cpu_base = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                     "frames_per_s": fr / t,
-                    "sample": f"first {nu} of {n_seq} utterances ({fr} frames; block + window oracle, "
-                              f"{t:.1f} s, fp64, {threads} threads), {cpu_info()}"}
+                    "sample": f"{nu} whole utterances of the {n_seq}-utterance batch, in order, wrapping "
+                              f"({fr} frames; block + window oracle, {t:.1f} s, fp64, {threads} threads), "
+                              f"{cpu_info()}"}
 
     hbm_peak, tf_peak, tf_sust, peak_src = measured_peaks()
     achieved_gbs = by_blk / (t_blk * 1e-3) / 1e9
-    traffic = None
-    if NCU_TRAFFIC["source_sha256"] == kernel_source_sha() and NCU_TRAFFIC["traffic_over_algorithmic"]:
-        traffic = NCU_TRAFFIC["traffic_over_algorithmic"] * by_blk
+    traffic = ncu_traffic("block_attn", by_blk)
     blk_tflops = f_blk / (t_blk * 1e-3) / 1e12
     value = world * flops_step / (ms_step * 1e-3) / 1e12
     line = {
@@ -386,7 +400,8 @@ def run_nle(args, rank, world, local):
                        "attainable_tflops": min(tf_peak, f_blk / by_blk * hbm_peak / 1e3),
                        "ai_flop_per_byte": f_blk / by_blk},
         "window_xattn": {"gbs": by_win / (t_win * 1e-3) / 1e9, "ms": t_win, "tflops": f_win / (t_win * 1e-3) / 1e12,
-                         "pct_of_hbm_peak": 100.0 * by_win / (t_win * 1e-3) / 1e9 / hbm_peak},
+                         "pct_of_hbm_peak": 100.0 * by_win / (t_win * 1e-3) / 1e9 / hbm_peak,
+                         "algorithmic_bytes": by_win, "traffic": ncu_traffic("window_xattn", by_win)},
         "roofline": {"kernel": "block_attn_kernel", "bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
                      "unit": "GB/s", "frac": achieved_gbs / hbm_peak, "traffic": traffic,
                      "algorithmic_bytes": by_blk, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},

@@ -571,6 +571,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = n % p.sqk, sv = n % kSV;
                 const uint32_t ph_qk = (uint32_t)(n / p.sqk) & 1, ph_v = (uint32_t)(n / kSV) & 1;
                 if (t == 1 && sL <= kQTile) {
+                    // no rows in slot 1: release its share of the stages.
+                    // v_ready (not v_full) is waited on, as for the blocks
+                    // slot 1 computes, so that slot 1 meets every phase of
+                    // v_ready in order and is never two phases ahead of it
+                    // (a parity wait on a phase that has not begun would
+                    // return at once).
                     if (leader) {
                         if (!wait_bar(smem_u32(&bars->qk_full[s]), ph_qk, abort_flag, wait_ns, p.status)) {
                             ok = false;
@@ -578,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         if (lane == 0)
                             mbar_arrive(smem_u32(&bars->qk_empty[s]));
-                        if (!wait_bar(smem_u32(&bars->v_full[sv]), ph_v, abort_flag, wait_ns, p.status)) {
+                        if (!wait_bar(smem_u32(&bars->v_ready[sv]), ph_v, abort_flag, wait_ns, p.status)) {
                             ok = false;
                             return false;
                         }

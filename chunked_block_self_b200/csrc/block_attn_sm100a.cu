@@ -8,34 +8,39 @@
 //     O = softmax(scale * Q K^T) V  over the block's L <= B frames.
 //
 // Design (one persistent CTA per SM, three warpgroups):
-//   warp 0      TMA producer.  Work item = (block, head).  Q (two boxes:
-//               rows 0..127 and 128..B-1), K and V of the item are loaded
-//               with 128-byte-swizzled TMA boxes (no multicast) into a ring
-//               of QK stages and a ring of two V stages; V lags QK by one
-//               item so Q/K run up to (stages) items ahead.
-//   warp 1      owns TMEM (allocates and frees it); warps 1-3 do no work.
-//   warps 4-7   tile slot 0 (block rows 0..127), warps 8-11 tile slot 1
-//               (rows 128..B-1, blocks longer than 128 frames).  The first
-//               warp of each warpgroup issues the slot's MMAs (one elected
-//               lane, warp-uniform descriptors):
-//                 S_t = Q_t K^T   tcgen05.mma kind::f16, M=128, N=ceil16(L),
+//   warps 0, 1  TMA producers.  Work item = (block, head).  Warp 0 loads
+//               Q (two boxes: rows 0..127 and 128..B-1) and K of each item
+//               into a ring of QK stages, warp 1 loads V into a ring of V
+//               stages, all as 128-byte-swizzled TMA boxes (no multicast).
+//               Warp 1 also owns TMEM (allocates and frees it).
+//   warps 4-7   tile warpgroup 0, TMEM slot 0: the CTA's even items,
+//   warps 8-11  tile warpgroup 1, TMEM slot 1: the odd items.  For each of
+//               its items a warpgroup computes row tile 0 (block rows
+//               0..127) and then, for blocks longer than 128 frames, row
+//               tile 1 (rows 128..B-1) in its slot; the two warpgroups run
+//               independent chains, so one's MMA and output phases overlap
+//               the other's softmax.  The first warp of each warpgroup
+//               issues the slot's MMAs (one elected lane, warp-uniform
+//               descriptors):
+//                 S = Q_x K^T     tcgen05.mma kind::f16, M=128, N=ceil16(L),
 //                                 K=64 in 4 steps
-//                 O_t = P_t V     A operand = P in TMEM, B = V (N-major) in
+//                 O_x = P V       A operand = P in TMEM, B = V (N-major) in
 //                                 smem, M=128, N=64, K=ceil16(L) in steps
 //                                 of 16
-//               Before PV of a partial block warpgroup 0 zeroes V rows
-//               L..ceil16(L)-1 in shared memory (frames outside the block;
-//               P is 0 there, but 0 * Inf would be NaN).  Each
+//               Before the first PV of a partial block the warpgroup zeroes
+//               V rows L..ceil16(L)-1 in shared memory (frames outside the
+//               block; P is 0 there, but 0 * Inf would be NaN).  Each
 //               thread owns one block row (its TMEM lane) and reads S in
 //               64-column register segments: p = exp2(S*scale*log2e
 //               - m) in fp32 with one shift m per row (keys >= L are 0 by
 //               index, never by value), row sum, bf16 pack, P written back
-//               over S.  The epilogue reads O, divides by
-//               the row sum and rounds to bf16; a warp whose 32 rows all lie
-//               in the block stages them (128-byte swizzle) in shared memory
-//               and writes them with one TMA store, otherwise its rows < L are
-//               written with 16-byte vector stores.  Rows past the block end
-//               are never written.
+//               over S.  The epilogue reads O, divides by the row sum,
+//               rounds to bf16 and writes each row < L with 16-byte vector
+//               stores, while the warpgroup's next S MMA runs.  Rows past the
+//               block end are never written.
+//               QK and V rings have even depths, so an item's stages have
+//               the parity of its warpgroup and each stage belongs to one
+//               warpgroup.
 // The MMAs of an item stop at ceil16(L) keys, so a partial block costs only
 // its own keys.
 // TMEM (512 columns): tile slot t at column 256*t holds S (NB columns), then
@@ -73,16 +78,9 @@ namespace {
 
 using namespace nle;
 
-// Three warpgroups: warp 0 producer, warp 1 TMEM owner, warps 2-3 idle,
+// Three warpgroups: warps 0-1 producers (warp 1 also owns TMEM), warps 2-3 idle,
 // warps 4-11 the two tile warpgroups (168 registers each; the softmax works
 // on 64-column segments of S).
-// The two tile warpgroups may take turns on the softmax (a token passed
-// through shared memory); by default they overlap, which keeps two softmax
-// warps per SM sub-partition and measured faster.
-#ifndef NLE_PINGPONG
-#define NLE_PINGPONG 0
-#endif
-constexpr bool kPingPong = NLE_PINGPONG != 0;
 constexpr int kThreads = 384;
 constexpr int kSoftmax0 = 4;
 constexpr int kSeg = 64;
@@ -90,25 +88,23 @@ constexpr int kSeg = 64;
 constexpr int kQTile = 128;        // MMA M (rows per tile)
 constexpr int kRowBytes = 128;     // one frame of one head: 64 bf16
 constexpr int kMaxQK = 4;          // QK ring depth upper bound
-constexpr int kSV = 2;             // V ring depth
+constexpr int kMaxV = 4;           // V ring depth upper bound
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256; // TMEM columns per tile slot
 constexpr uint32_t kOCol = 128;     // O offset inside a tile slot
 
 struct Bars {
     uint64_t qk_full[kMaxQK];
-    uint64_t qk_empty[kMaxQK];   // 2 arrivals: the two tile warpgroups
-    uint64_t v_full[kSV];
-    uint64_t v_ready[kSV];       // tail rows of a partial block zeroed
-    uint64_t v_empty[kSV];       // 2 arrivals: the two tile warpgroups
+    uint64_t qk_empty[kMaxQK];   // the item's last S MMA has completed
+    uint64_t v_full[kMaxV];
+    uint64_t v_empty[kMaxV];     // the item's last PV MMA has completed
     uint64_t s_full[2];
-    uint64_t wg_p[2];            // 4 arrivals: P of the tile written
+    uint64_t wg_p[2];            // 4 arrivals: P of the unit written
     uint64_t o_full[2];
-    uint64_t wg_o[2];            // 4 arrivals: O of the tile read from TMEM
+    uint64_t wg_o[2];            // 4 arrivals: O of the unit read from TMEM
     uint64_t mma_done[2];
     uint32_t tmem_base;
     int abort_flag;
-    int turn;                    // softmax phases completed (ping-pong token)
 };
 
 struct Params {
@@ -120,11 +116,11 @@ struct Params {
     int q0rows;   // rows of the first Q box (min(B, 128))
     int q1rows;   // rows of the second Q box (B - 128, or 0)
     int sqk;      // QK ring depth
+    int nsv;      // V ring depth
     uint32_t q_bytes;   // Q region of a QK stage
     uint32_t qk_bytes;  // QK stage
     uint32_t v_bytes;   // V stage
-    uint32_t stage_off; // output staging: stage_bufs x 4 KB per softmax warp
-    int stage_bufs;     // 2 (alternating) when shared memory allows, else 1
+    uint32_t bars_off;  // barriers, after the QK and V rings
     float scale_log2;
     __nv_bfloat16 *out;
     int out_stride;     // elements between output frames (heads * 64)
@@ -373,15 +369,14 @@ __device__ __forceinline__ float softmax_rows(uint32_t tS, int L, float sl2, int
 template <int NB>
 __global__ void __launch_bounds__(kThreads, 1)
     block_attn_kernel(const __grid_constant__ CUtensorMap tm_q0, const __grid_constant__ CUtensorMap tm_q1,
-                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_o, const Params p)
+                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t qk_base = smem_u32(smem);
     const uint32_t v_off = p.sqk * p.qk_bytes;
     const uint32_t v_base = qk_base + v_off;
-    Bars *bars = reinterpret_cast<Bars *>(smem + p.stage_off + 8 * p.stage_bufs * 4096);
+    Bars *bars = reinterpret_cast<Bars *>(smem + p.bars_off);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -389,12 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.sqk; ++s) {
             mbar_init(smem_u32(&bars->qk_full[s]), 1);
-            mbar_init(smem_u32(&bars->qk_empty[s]), 2);
+            mbar_init(smem_u32(&bars->qk_empty[s]), 1);
         }
-        for (int s = 0; s < kSV; ++s) {
+        for (int s = 0; s < p.nsv; ++s) {
             mbar_init(smem_u32(&bars->v_full[s]), 1);
-            mbar_init(smem_u32(&bars->v_ready[s]), 1);
-            mbar_init(smem_u32(&bars->v_empty[s]), 2);
+            mbar_init(smem_u32(&bars->v_empty[s]), 1);
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(smem_u32(&bars->s_full[t]), 1);
@@ -404,7 +398,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&bars->mma_done[t]), 1);
         }
         bars->abort_flag = 0;
-        bars->turn = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -416,12 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_q1);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
-        tma_prefetch_desc(&tm_o);
     }
     // V rows B..NB-1 (MMA padding) are zero for the whole launch.
     {
         const int pad_chunks = (NB - p.B) * (kRowBytes / 16);
-        for (int i = threadIdx.x; i < kSV * pad_chunks; i += kThreads) {
+        for (int i = threadIdx.x; i < p.nsv * pad_chunks; i += kThreads) {
             const int s = i / pad_chunks, c = i - s * pad_chunks;
             reinterpret_cast<uint4 *>(smem + v_off + s * p.v_bytes + p.B * kRowBytes)[c] = make_uint4(0, 0, 0, 0);
         }
@@ -438,45 +430,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int step_b = (int)(gridDim.x / H), step_h = (int)(gridDim.x % H);
     const int first_b = (int)(blockIdx.x / H), first_h = (int)(blockIdx.x % H);
 
-    if (warp < kSoftmax0) {
-        if (warp == 0) {
-            // ==================================================== producer
-            PlanWalker w;
-            w.init(p.cu, p.n_seq, p.total, p.B, lane);
-            const uint64_t pol = policy_evict_first();
-            int qk_count = 0, v_count = 0;   // copies issued (stages used round-robin)
-            int prev_h = 0, prev_f0 = 0;
-            int n = 0;
-            bool ok = true;
-
-            auto issue_v = [&](int m, int h, int f0) -> bool {
-                const int sv = m % kSV;
-                const uint32_t uv = (uint32_t)(m / kSV);
-                if (uv > 0 &&
-                    !wait_bar(smem_u32(&bars->v_empty[sv]), (uv - 1) & 1, abort_flag, wait_ns, p.status))
-                    return false;
-                if (lane == 0) {
-                    const uint32_t bar = smem_u32(&bars->v_full[sv]);
+    if (warp == 0 || warp == 1) {
+        // ==================================================== producers
+        // Warp 0 loads Q and K of every item, warp 1 loads V; each refills a
+        // stage as soon as the stage's last reader has released it (QK: the
+        // item's last S MMA; V: its last PV MMA).
+        const bool is_v = warp == 1;
+        const int nst = is_v ? p.nsv : p.sqk;
+        PlanWalker w;
+        w.init(p.cu, p.n_seq, p.total, p.B, lane);
+        const uint64_t pol = policy_evict_first();
+        const bool skip0 = !is_v && (p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) != 0;
+        int n = 0;   // items whose copies were issued
+        for (int b = first_b, h = first_h;; ++n) {
+            int f0, L, seq;
+            if (!w.find(b, lane, f0, L, seq))
+                break;
+            const int s = n % nst;
+            const uint32_t u = (uint32_t)(n / nst);
+            if (u > 0 && !wait_bar(smem_u32(is_v ? &bars->v_empty[s] : &bars->qk_empty[s]), (u - 1) & 1, abort_flag,
+                                   wait_ns, p.status))
+                break;
+            if (lane == 0) {
+                if (is_v) {
+                    const uint32_t bar = smem_u32(&bars->v_full[s]);
                     mbar_arrive_expect_tx(bar, p.B * kRowBytes);
-                    tma_load_2d(v_base + sv * p.v_bytes, &tm_v, h * 64, f0, bar, pol);
-                }
-                ++v_count;
-                __syncwarp();
-                return true;
-            };
-
-            for (int b = first_b, h = first_h;; ++n) {
-                int f0, L, seq;
-                if (!w.find(b, lane, f0, L, seq))
-                    break;
-                const int s = n % p.sqk;
-                const uint32_t u = (uint32_t)(n / p.sqk);
-                if (u > 0 &&
-                    !wait_bar(smem_u32(&bars->qk_empty[s]), (u - 1) & 1, abort_flag, wait_ns, p.status)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0 && !((p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) && n == 0)) {
+                    tma_load_2d(v_base + s * p.v_bytes, &tm_v, h * 64, f0, bar, pol);
+                } else if (!(skip0 && n == 0)) {
                     const bool two = L > kQTile;
                     const uint32_t bar = smem_u32(&bars->qk_full[s]);
                     const uint32_t bytes = (p.q0rows + (two ? p.q1rows : 0) + p.B) * kRowBytes;
@@ -487,197 +467,141 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d(qdst + kQTile * kRowBytes, &tm_q1, h * 64, f0 + kQTile, bar, pol);
                     tma_load_2d(qdst + p.q_bytes, &tm_k, h * 64, f0, bar, pol);
                 }
-                ++qk_count;
-                __syncwarp();
-                if (n > 0 && !issue_v(n - 1, prev_h, prev_f0)) {
-                    ok = false;
-                    break;
-                }
-                prev_h = h;
-                prev_f0 = f0;
-                b += step_b;
-                h += step_h;
-                if (h >= H) {
-                    h -= H;
-                    ++b;
-                }
-            }
-            if (ok && n > 0)
-                issue_v(n - 1, prev_h, prev_f0);
-            if (w.bad && lane == 0)
-                report(p.status, NLE_ERR_INVALID_ARG);
-            // drain: every issued copy must land before the CTA can exit.
-            // Copies went to stages round-robin, so the last ones to each
-            // stage are those of the final min(count, stages) items.
-            if (lane == 0) {
-                const bool skipped0 = (p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) != 0;
-                for (int m = qk_count - p.sqk; m < qk_count; ++m)
-                    if (m >= 0 && !(skipped0 && m == 0))
-                        wait_bar_drain(smem_u32(&bars->qk_full[m % p.sqk]), (uint32_t)(m / p.sqk) & 1, wait_ns);
-                for (int m = v_count - kSV; m < v_count; ++m)
-                    if (m >= 0)
-                        wait_bar_drain(smem_u32(&bars->v_full[m % kSV]), (uint32_t)(m / kSV) & 1, wait_ns);
+                NLE_TRACE_AT(0, n, is_v ? 1 : 0);
             }
             __syncwarp();
+            b += step_b;
+            h += step_h;
+            if (h >= H) {
+                h -= H;
+                ++b;
+            }
         }
+        if (!is_v && w.bad && lane == 0)
+            report(p.status, NLE_ERR_INVALID_ARG);
+        // drain: every issued copy must land before the CTA can exit.
+        // Copies went to stages round-robin, so the last ones to each stage
+        // are those of the final min(n, stages) items.
+        if (lane == 0) {
+            for (int m = n - nst; m < n; ++m)
+                if (m >= 0 && !(skip0 && m == 0))
+                    wait_bar_drain(smem_u32(is_v ? &bars->v_full[m % nst] : &bars->qk_full[m % nst]),
+                                   (uint32_t)(m / nst) & 1, wait_ns);
+        }
+        __syncwarp();
+    } else if (warp < kSoftmax0) {
+        // warps 2, 3: no role
     } else {
         // ======================================================== tile warpgroups
-        // Warpgroup t drives TMEM slot t: its first warp's elected lane
-        // issues the slot's MMAs, all four warps run softmax and epilogue.
-        // The two warpgroups take turns on the softmax (the MUFU-bound
-        // phase): one runs it while the other waits on its MMAs or writes
-        // its output.  The turn order is block by block, slot 0 then slot 1.
-        const int t = (warp - kSoftmax0) >> 2;     // tile slot
+        // Warpgroup t owns TMEM slot t and computes the CTA's items
+        // n = t, t + 2, t + 4, ...: for each, row tile 0 (block rows
+        // 0..127) and then, for blocks longer than 128 frames, row tile 1
+        // (rows 128..B-1), one after the other in its slot.  The two
+        // warpgroups thus run independent chains, and one's MMA and output
+        // phases overlap the other's softmax.  The first warp's elected lane
+        // issues the slot's MMAs; all four warps run softmax and epilogue.
+        const int t = (warp - kSoftmax0) >> 2;     // TMEM slot
         const int qq = warp & 3;                   // TMEM lane quarter of this warp
         const bool leader = qq == 0;
         const uint32_t slot = tmem + t * kSlotCols;
         const uint32_t tS = slot + ((uint32_t)(qq * 32) << 16);
         const float sl2 = p.scale_log2;
         const uint32_t id_pv = idesc_bf16_f32(128, 64, true);
-        // output staging of this warp: two buffers of 32 rows x 128 B,
-        // 128-byte swizzle
-        const uint32_t stage_u32 = smem_u32(smem + p.stage_off + (warp - kSoftmax0) * p.stage_bufs * 4096);
-        int stores = 0;
         PlanWalker w;
         w.init(p.cu, p.n_seq, p.total, p.B, lane);
-        volatile int *turn = &bars->turn;
+        // the CTA's item sequence: item n is blockIdx.x + n * gridDim.x
         int b = first_b, h = first_h;
-        int n = -1;          // index of the current block among this CTA's items
-        int c1 = 0;          // blocks seen so far that have rows in slot 1
-        uint32_t uses = 0;   // blocks this slot has computed
-        int f0 = 0, L = 0, hcur = 0, my_turn = 0, nkeys = 16;
+        int next_n = 0;      // next item of the CTA's sequence (not yet looked at)
+        int n = -1;          // current item
+        int x = 1;           // current row tile of the item
+        uint32_t uses = 0;   // units (item, row tile) this slot has computed
+        int f0 = 0, L = 0, hcur = 0, nkeys = 16, s = 0, sv = 0;
         bool ok = true;
 
-        // Advance to the next block with rows in this slot; on the way,
-        // slot 1 releases its share of the stages of blocks it skips.  The
-        // leader then issues the block's S MMA (after the slot's previous O
-        // has been read by all four warps).  False at the end of the work.
+        // Move to the slot's next unit: row tile 1 of the current item if it
+        // has one, else row tile 0 of the slot's next item.  The leader then
+        // issues the unit's S MMA (after the slot's previous O has been read
+        // by all four warps).  False at the end of the work.
+        // Both ring depths are even, so the item's stages have the parity of
+        // its slot: each stage belongs to one slot, whose items meet its
+        // phases one by one, in order (a parity wait is only meaningful on
+        // the current phase or the one after it).
         auto advance = [&]() -> bool {
-            for (;;) {
-                int sf0, sL, sseq;
-                if (!w.find(b, lane, sf0, sL, sseq))
-                    return false;
-                ++n;
-                const int hh = h;
-                b += step_b;
-                h += step_h;
-                if (h >= H) {
-                    h -= H;
-                    ++b;
-                }
-                const int c1_before = c1;
-                if (sL > kQTile)
-                    ++c1;
-                const int s = n % p.sqk, sv = n % kSV;
-                const uint32_t ph_qk = (uint32_t)(n / p.sqk) & 1, ph_v = (uint32_t)(n / kSV) & 1;
-                if (t == 1 && sL <= kQTile) {
-                    // no rows in slot 1: release its share of the stages.
-                    // v_ready (not v_full) is waited on, as for the blocks
-                    // slot 1 computes, so that slot 1 meets every phase of
-                    // v_ready in order and is never two phases ahead of it
-                    // (a parity wait on a phase that has not begun would
-                    // return at once).
-                    if (leader) {
-                        if (!wait_bar(smem_u32(&bars->qk_full[s]), ph_qk, abort_flag, wait_ns, p.status)) {
-                            ok = false;
-                            return false;
-                        }
-                        if (lane == 0)
-                            mbar_arrive(smem_u32(&bars->qk_empty[s]));
-                        if (!wait_bar(smem_u32(&bars->v_ready[sv]), ph_v, abort_flag, wait_ns, p.status)) {
-                            ok = false;
-                            return false;
-                        }
-                        if (lane == 0)
-                            mbar_arrive(smem_u32(&bars->v_empty[sv]));
+            if (!(x == 0 && L > kQTile)) {
+                // the slot's next item: pass over the other slot's one
+                for (;;) {
+                    int sf0, sL, sseq;
+                    if (!w.find(b, lane, sf0, sL, sseq))
+                        return false;
+                    const int nn = next_n++;
+                    const int hh = h;
+                    b += step_b;
+                    h += step_h;
+                    if (h >= H) {
+                        h -= H;
+                        ++b;
                     }
-                    continue;
+                    if ((nn & 1) != t)
+                        continue;
+                    n = nn;
+                    f0 = sf0;
+                    L = sL;
+                    hcur = hh;
+                    break;
                 }
-                f0 = sf0;
-                L = sL;
-                hcur = hh;
+                x = 0;
                 nkeys = (L + 15) & ~15;   // MMA extent over keys
-                my_turn = n + c1_before + t;
-                if (leader) {
-                    if (lane == 0)
-                        NLE_TRACE_AT(1 + t, n, 0);
-                    if (!wait_bar(smem_u32(&bars->qk_full[s]), ph_qk, abort_flag, wait_ns, p.status)) {
-                        ok = false;
-                        return false;
-                    }
-                    if (lane == 0)
-                        NLE_TRACE_AT(1 + t, n, 1);
-                    if (uses > 0 &&
-                        !wait_bar(smem_u32(&bars->wg_o[t]), (uses - 1) & 1, abort_flag, wait_ns, p.status)) {
-                        ok = false;
-                        return false;
-                    }
-                    tc_fence_after();
-                    if (lane == 0)
-                        NLE_TRACE_AT(1 + t, n, 2);
-                    // K steps of 16 elements = 32 bytes inside the 128-byte
-                    // swizzle atom: advance the descriptor start address
-                    const uint32_t qaddr = qk_base + s * p.qk_bytes;
-                    const uint64_t da = smem_desc_sw128(qaddr + t * kQTile * kRowBytes, 16, 1024);
-                    const uint64_t db = smem_desc_sw128(qaddr + p.q_bytes, 16, 1024);
-                    const uint32_t id_s = idesc_bf16_f32(128, nkeys, false);
-                    if (elect_one()) {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ss(slot, da + 2 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
-                        mma_commit(smem_u32(&bars->s_full[t]));
-                        mma_commit(smem_u32(&bars->qk_empty[s]));
-                        NLE_TRACE_AT(1 + t, n, 3);
-                    }
-                    __syncwarp();
-                }
-                return true;
+                s = n % p.sqk;
+                sv = n % p.nsv;
+            } else {
+                x = 1;
             }
+            if (leader) {
+                if (lane == 0)
+                    NLE_TRACE_AT(1 + t, n * 2 + x, 0);
+                if (x == 0 &&
+                    !wait_bar(smem_u32(&bars->qk_full[s]), (uint32_t)(n / p.sqk) & 1, abort_flag, wait_ns, p.status)) {
+                    ok = false;
+                    return false;
+                }
+                if (uses > 0 &&
+                    !wait_bar(smem_u32(&bars->wg_o[t]), (uses - 1) & 1, abort_flag, wait_ns, p.status)) {
+                    ok = false;
+                    return false;
+                }
+                tc_fence_after();
+                // K steps of 16 elements = 32 bytes inside the 128-byte
+                // swizzle atom: advance the descriptor start address
+                const uint32_t qaddr = qk_base + s * p.qk_bytes;
+                const uint64_t da = smem_desc_sw128(qaddr + x * kQTile * kRowBytes, 16, 1024);
+                const uint64_t db = smem_desc_sw128(qaddr + p.q_bytes, 16, 1024);
+                const uint32_t id_s = idesc_bf16_f32(128, nkeys, false);
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(slot, da + 2 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
+                    mma_commit(smem_u32(&bars->s_full[t]));
+                    if (x == 1 || L <= kQTile)   // the item's last S: its QK stage can be reused
+                        mma_commit(smem_u32(&bars->qk_empty[s]));
+                    NLE_TRACE_AT(1 + t, n * 2 + x, 1);
+                }
+                __syncwarp();
+            }
+            return true;
         };
 
-        // Each pass: advance (the leader issues the next block's S MMA),
-        // write the previous block's output, then compute the current block.
+        // Each pass: advance (the leader issues the next unit's S MMA),
+        // write the previous unit's output, then compute the current unit.
         uint32_t pk[32];
-        bool pending = false;          // pk holds rows of the previous block
+        bool pending = false;          // pk holds rows of the previous unit
         int ef0 = 0, eL = 0, eh = 0, erow0 = 0;
         for (;;) {
             const bool have = advance();
             if (!ok)
                 break;
             if (pending) {
-                if (erow0 + 32 <= eL) {
-                    // all 32 rows inside the block: stage (swizzled) and
-                    // store with one TMA box of 32 rows; two staging buffers
-                    // alternate
-                    const uint32_t buf = stage_u32 + (stores % p.stage_bufs) * 4096;
-                    if (stores >= p.stage_bufs) {
-                        // the store that used this buffer must have read it
-                        if (lane == 0) {
-                            if (p.stage_bufs == 2)
-                                bulk_wait_read1();
-                            else
-                                bulk_wait_read0();
-                        }
-                        __syncwarp();
-                    }
-                    // the row's base address is made opaque here so the
-                    // eight swizzled addresses are formed at the stores, not
-                    // hoisted out of the block loop
-                    uint32_t srow = buf + lane * 128;
-                    asm volatile("" : "+r"(srow));
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        st_shared_v4(srow + ((c ^ (lane & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                                     pk[4 * c + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tm_o, eh * 64, ef0 + erow0, buf);
-                        bulk_commit();
-                    }
-                    ++stores;
-                } else if (erow0 + lane < eL) {
-                    // rows past the block end are never written
+                // rows past the block end are never written
+                if (erow0 + lane < eL) {
                     uint4 *dst =
                         reinterpret_cast<uint4 *>(p.out + (size_t)(ef0 + erow0 + lane) * p.out_stride + eh * 64);
 #pragma unroll
@@ -688,53 +612,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!have)
                 break;
-            const int sv = n % kSV;
-            const uint32_t ph_v = (uint32_t)(n / kSV) & 1;
+            const uint32_t ph_v = (uint32_t)(n / p.nsv) & 1;
             // ---------------------------------------------- softmax
             if (!wait_bar(smem_u32(&bars->s_full[t]), uses & 1, abort_flag, wait_ns, p.status))
                 break;
             tc_fence_after();
-            // wait for this slot's turn on the softmax (bounded)
-            if (kPingPong && *turn < my_turn) {
-                const uint64_t t0 = globaltimer_ns();
-                while (*turn < my_turn) {
-                    __nanosleep(32);
-                    if (*abort_flag) {
-                        ok = false;
-                        break;
-                    }
-                    if (globaltimer_ns() - t0 > wait_ns) {
-                        *abort_flag = 1;
-                        report(p.status, NLE_ERR_TIMEOUT);
-                        ok = false;
-                        break;
-                    }
-                }
-                if (!__all_sync(kFull, ok))
-                    break;
-            }
             if (lane == 0 && qq == 0)
-                NLE_TRACE_AT(3 + t, n, 0);
-            const int row0 = t * kQTile + qq * 32;   // first block row of this warp
+                NLE_TRACE_AT(3 + t, n * 2 + x, 0);
+            const int row0 = x * kQTile + qq * 32;   // first block row of this warp
             const bool active = row0 < L;
             float l = 1.f;
             if (active)
-                l = softmax_rows<NB, kSeg>(tS, L, sl2, (lane == 0 && qq == 0) ? 3 + t : -1, n);
+                l = softmax_rows<NB, kSeg>(tS, L, sl2, (lane == 0 && qq == 0) ? 3 + t : -1, n * 2 + x);
             if (lane == 0 && qq == 0)
-                NLE_TRACE_AT(3 + t, n, 1);
-            if (t == 0 && L < nkeys && L < p.B) {
-                // PV reads V rows 0..nkeys-1; rows L..nkeys-1 of a partial
-                // block hold frames of the next block (or utterance): zero
-                // them so nothing outside the block reaches PV (P is 0 there,
-                // but 0 * Inf would be NaN).  Rows B..NB-1 are always zero.
-                if (!wait_bar(smem_u32(&bars->v_full[sv]), ph_v, abort_flag, wait_ns, p.status))
-                    break;
-                const int zend = nkeys < p.B ? nkeys : p.B;
-                uint4 *vz = reinterpret_cast<uint4 *>(smem + v_off + sv * p.v_bytes + L * kRowBytes);
-                for (int i = qq * 32 + lane; i < (zend - L) * (kRowBytes / 16); i += 128)
-                    vz[i] = make_uint4(0, 0, 0, 0);
-                fence_proxy_async_smem();
-            }
+                NLE_TRACE_AT(3 + t, n * 2 + x, 1);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -743,19 +634,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) {
                 if (!wait_bar(smem_u32(&bars->wg_p[t]), uses & 1, abort_flag, wait_ns, p.status))
                     break;
-                if (lane == 0)
-                    *turn = my_turn + 1;   // the other slot may run its softmax
-                if (t == 0) {
+                if (x == 0) {
                     if (!wait_bar(smem_u32(&bars->v_full[sv]), ph_v, abort_flag, wait_ns, p.status))
                         break;
-                    if (lane == 0)
-                        mbar_arrive(smem_u32(&bars->v_ready[sv]));   // tail rows zeroed
-                } else if (!wait_bar(smem_u32(&bars->v_ready[sv]), ph_v, abort_flag, wait_ns, p.status)) {
-                    break;
+                    if (L < nkeys && L < p.B) {
+                        // PV reads V rows 0..nkeys-1; rows L..nkeys-1 of a
+                        // partial block hold frames of the next block (or
+                        // utterance): zero them so nothing outside the block
+                        // reaches PV (P is 0 there, but 0 * Inf would be
+                        // NaN).  Rows B..NB-1 are always zero.
+                        const int zend = nkeys < p.B ? nkeys : p.B;
+                        uint4 *vz = reinterpret_cast<uint4 *>(smem + v_off + sv * p.v_bytes + L * kRowBytes);
+                        for (int i = lane; i < (zend - L) * (kRowBytes / 16); i += 32)
+                            vz[i] = make_uint4(0, 0, 0, 0);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
                 }
                 tc_fence_after();
                 if (lane == 0)
-                    NLE_TRACE_AT(1 + t, n, 5);
+                    NLE_TRACE_AT(1 + t, n * 2 + x, 5);
                 // N = 64 is one 128-byte swizzle atom along N, so the
                 // N-direction atom stride (LBO) is never used; K steps of 16
                 // rows advance the start address by 2048 bytes.
@@ -765,8 +663,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_ts(slot + kOCol, slot + kk * 8, dv + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
                                kk > 0 ? 1u : 0u);
                     mma_commit(smem_u32(&bars->o_full[t]));
-                    mma_commit(smem_u32(&bars->v_empty[sv]));
-                    NLE_TRACE_AT(1 + t, n, 6);
+                    if (x == 1 || L <= kQTile)   // the item's last PV: its V stage can be reused
+                        mma_commit(smem_u32(&bars->v_empty[sv]));
+                    NLE_TRACE_AT(1 + t, n * 2 + x, 6);
                 }
                 __syncwarp();
             }
@@ -775,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             tc_fence_after();
             if (lane == 0 && qq == 0)
-                NLE_TRACE_AT(3 + t, n, 2);
+                NLE_TRACE_AT(3 + t, n * 2 + x, 2);
             if (active) {
                 uint32_t o[64];
 #pragma unroll
@@ -795,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0)
                 mbar_arrive(smem_u32(&bars->wg_o[t]));
             if (lane == 0 && qq == 0)
-                NLE_TRACE_AT(3 + t, n, 3);
+                NLE_TRACE_AT(3 + t, n * 2 + x, 3);
             ++uses;
             pending = active;
             ef0 = f0;
@@ -803,9 +702,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             eh = hcur;
             erow0 = row0;
         }
-        if (lane == 0 && stores > 0)
-            bulk_wait0();
-        __syncwarp();
         // this slot's MMAs must finish before TMEM is released
         if (leader) {
             if (elect_one()) {
@@ -825,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-using BlockKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, Params);
+using BlockKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, Params);
 
 struct KernelInfo {
     BlockKernel fn;
@@ -912,21 +808,28 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
     p.q_bytes = (uint32_t)((rows8 > kQTile ? rows8 : kQTile) * kRowBytes);
     p.qk_bytes = p.q_bytes + (uint32_t)(rows8 * kRowBytes);
     p.v_bytes = (uint32_t)(NB * kRowBytes);
-    // fixed part: V ring, output staging (per softmax warp 2 x 4 KB, or
-    // 4 KB when that would leave fewer than two QK stages), barriers,
-    // alignment slack
-    const size_t other = (size_t)kSV * p.v_bytes + ((sizeof(Bars) + 127) / 128) * 128 + 1024;
-    p.stage_bufs = 2;
-    if ((size_t)di.smem_optin < other + (size_t)8 * 8192 + 2 * (size_t)p.qk_bytes)
-        p.stage_bufs = 1;
-    const size_t fixed = other + (size_t)8 * 4096 * p.stage_bufs;
-    int sqk = (int)(((size_t)di.smem_optin - fixed) / p.qk_bytes);
-    if (sqk > kMaxQK)
-        sqk = kMaxQK;
-    if (sqk < 2)
+    // Shared memory: QK ring and V ring, each of an even depth (the two
+    // tile warpgroups take alternate items, so each stage then belongs to
+    // one warpgroup), as deep as fits (V first: it is held from the item's
+    // first PV to its last), then the barriers and alignment slack.
+    const size_t bars_bytes = ((sizeof(Bars) + 127) / 128) * 128 + 1024;
+    int sqk = 0, nsv = 0;
+    for (const int v : {4, 2}) {
+        for (const int q : {4, 2})
+            if ((size_t)q * p.qk_bytes + (size_t)v * p.v_bytes + bars_bytes <= (size_t)di.smem_optin) {
+                sqk = q;
+                nsv = v;
+                break;
+            }
+        if (sqk)
+            break;
+    }
+    if (!sqk)
         return NLE_ERR_UNSUPPORTED;
     p.sqk = sqk;
-    p.stage_off = (uint32_t)(sqk * p.qk_bytes + kSV * p.v_bytes);
+    p.nsv = nsv;
+    p.bars_off = (uint32_t)(sqk * p.qk_bytes + nsv * p.v_bytes);
+    const size_t fixed = (size_t)nsv * p.v_bytes + bars_bytes;
     size_t smem = (size_t)sqk * p.qk_bytes + fixed;
     // One CTA per SM: it owns all 512 TMEM columns, so a second resident CTA
     // would only wait in tcgen05.alloc.  Ask for more than half the SM's
@@ -941,13 +844,12 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
     p.wait_ns = wait_limit_ns > 0 ? (unsigned long long)wait_limit_ns : 1000000000ull;
     p.flags = flags;
 
-    CUtensorMap tq0, tq1, tk, tv, to;
+    CUtensorMap tq0, tq1, tk, tv;
     const uint64_t cols = (uint64_t)dense, rows = (uint64_t)total_frames;
     if (!nle::encode_tmap_bf16_2d(&tq0, q, cols, rows, stride, 64, p.q0rows) ||
         !nle::encode_tmap_bf16_2d(&tq1, q, cols, rows, stride, 64, p.q1rows ? p.q1rows : p.q0rows) ||
         !nle::encode_tmap_bf16_2d(&tk, k, cols, rows, stride, 64, B) ||
-        !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, stride, 64, B) ||
-        !nle::encode_tmap_bf16_2d(&to, out, cols, rows, dense, 64, 32))
+        !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, stride, 64, B))
         return NLE_ERR_CUDA;
 
     const KernelInfo kern = pick_kernel(NB);
@@ -960,7 +862,7 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
         set = (int)smem;
     }
     const int grid = (int)(max_items < di.sm_count ? max_items : di.sm_count);
-    kern.fn<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tq0, tq1, tk, tv, to, p);
+    kern.fn<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tq0, tq1, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
 }
 

@@ -79,6 +79,24 @@ bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t cols, uint
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows][heads][64] bf16 (row stride `row_stride_elems`) viewed as a 3-D
+// tensor ordered (d, row, head), so that a box of (64, box_rows, box_heads)
+// lands in shared memory head-major: box_rows rows of 128 B per head.
+bool encode_tmap_bf16_heads(CUtensorMap *map, const void *base, uint64_t rows, uint64_t heads,
+                            uint64_t row_stride_elems, uint32_t box_rows, uint32_t box_heads)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[3] = {64, rows, heads};
+    const cuuint64_t strides[2] = {row_stride_elems * 2, 128};
+    const cuuint32_t box[3] = {64, box_rows, box_heads};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 } // namespace nle
 
 extern "C" int nle_version(void) { return NLE_ABI_VERSION; }

@@ -23,6 +23,11 @@ bool current_device_info(DeviceInfo *info, int *device);
 // 128-byte swizzle, zero fill outside the bounds.
 bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
                          uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
+// [rows][heads][64] bf16 as a 3-D tensor (d, row, head): boxes of
+// (64, box_rows, box_heads) land head-major in shared memory; 128-byte
+// swizzle, zero fill outside the tensor.
+bool encode_tmap_bf16_heads(CUtensorMap *map, const void *base, uint64_t rows, uint64_t heads,
+                            uint64_t row_stride_elems, uint32_t box_rows, uint32_t box_heads);
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

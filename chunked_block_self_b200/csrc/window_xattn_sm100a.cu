@@ -10,10 +10,12 @@
 //
 // The work is HBM-bound (about 2.5 flop per byte).  One persistent CTA per
 // SM walks windows g = blockIdx.x, blockIdx.x + gridDim.x, ...:
-//   warp 16     producer: per window one 128-byte-swizzled TMA box per head
-//               for K and for V (W rows of 64 bf16; no multicast) and one
-//               bulk copy for the window's contiguous query rows, into a
-//               ring of shared-memory stages.
+//   warp 16     producer: per window three 128-byte-swizzled TMA boxes (no
+//               multicast) into a ring of shared-memory stages: K and V of
+//               all heads (16 frames per 16-key group) and the window's Qw
+//               query rows of all heads, each through a 3-D tensor map
+//               ordered (d, row, head) so that every head's rows land
+//               together.
 //   warps 0-15  one head each (heads h = warp, warp + 16, ...): the window's
 //               S = Q K^T (at most 16 queries x 16 keys) and O = P V are
 //               warp-level mma.sync m16n8k16 products (bf16 in, fp32
@@ -39,6 +41,7 @@ constexpr int kThreads = (kComputeWarps + 1) * 32;
 constexpr int kMaxStages = 4;
 constexpr int kMaxQw = 16;
 constexpr int kTileBytes = 2048;   // 16 rows x 128 B, one head's keys (or values) per 16-key group
+constexpr int kOStride = 144;      // output staging row: 128 B + 16 B so fragment stores hit distinct banks
 
 struct WBars {
     uint64_t full[kMaxStages];
@@ -53,15 +56,14 @@ struct WParams {
     long long n_qrows;
     int heads;
     int W;        // window_frames
-    int box_rows; // rows of one K/V box: min(W, 16)
     int Qw;       // queries_per_window
     const __nv_bfloat16 *q;
     __nv_bfloat16 *out;
     int stages;
-    uint32_t kv_bytes;    // K (or V) region of a stage: heads * KT * 2048
-    uint32_t q_bytes;     // Q rows of a window: Qw * heads * 128
+    uint32_t kv_bytes;    // K (or V) region of a stage: KT * heads * 2048, [kt][head]
+    uint32_t q_bytes;     // Q rows of a window: heads * Qw * 128, [head][query]
     uint32_t stage_bytes;
-    uint32_t ostage_off;  // per-warp output staging (Qw x 128 B each)
+    uint32_t ostage_off;  // per-warp output staging (Qw rows of kOStride bytes)
     uint32_t bars_off;
     float scale_log2;
     int32_t *status;
@@ -102,7 +104,7 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 +
 template <int KT>
 __global__ void __launch_bounds__(kThreads, 1)
     window_xattn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                        const WParams p)
+                        const __grid_constant__ CUtensorMap tm_q, const WParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -123,21 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 32) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
-    }
-    // With one 16-key group (W <= 16), value rows W..15 of every head tile
-    // are MMA padding: never loaded, always zero (P is 0 there, and 0 * NaN
-    // would not be).  With two groups the boxes are 16 rows and rows past W
-    // are zeroed per window below.
-    if (KT == 1) {
-        const int pad_rows = 16 - p.W;
-        const int per_stage = H * KT * pad_rows * 8;   // 16-byte chunks
-        for (int i = threadIdx.x; i < p.stages * per_stage; i += kThreads) {
-            const int s = i / per_stage, r = i - s * per_stage;
-            const int tile = r / (pad_rows * 8), c = r - tile * pad_rows * 8;
-            uint8_t *vt = smem + s * p.stage_bytes + p.kv_bytes + tile * kTileBytes;
-            reinterpret_cast<uint4 *>(vt + (16 - pad_rows) * 128)[c] = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
+        tma_prefetch_desc(&tm_q);
     }
     __syncthreads();
     volatile int *abort_flag = &bars->abort_flag;
@@ -164,16 +152,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if ((long long)p.Qw * (g + 1) > p.n_qrows) {
                     mbar_arrive(bar);   // no query rows: consumers skip this window
                 } else {
-                    mbar_arrive_expect_tx(bar, 2u * H * KT * (uint32_t)p.box_rows * 128u + p.q_bytes);
-                    for (int h = 0; h < H; ++h) {
-                        for (int kt = 0; kt < KT; ++kt) {
-                            // one box of min(W, 16) rows per 16-key group
-                            tma_load_2d(st + (h * KT + kt) * kTileBytes, &tm_k, h * 64, f0 + 16 * kt, bar, pol);
-                            tma_load_2d(st + p.kv_bytes + (h * KT + kt) * kTileBytes, &tm_v, h * 64, f0 + 16 * kt,
-                                        bar, pol);
-                        }
+                    mbar_arrive_expect_tx(bar, 2u * p.kv_bytes + p.q_bytes);
+                    // 16 frames of every head per 16-key group (frames past
+                    // the window are masked, and zeroed in V, below)
+                    for (int kt = 0; kt < KT; ++kt) {
+                        tma_load_3d(st + kt * H * kTileBytes, &tm_k, 0, f0 + 16 * kt, 0, bar, pol);
+                        tma_load_3d(st + p.kv_bytes + kt * H * kTileBytes, &tm_v, 0, f0 + 16 * kt, 0, bar, pol);
                     }
-                    bulk_load(st + 2 * p.kv_bytes, p.q + (long long)p.Qw * g * row_elems, p.q_bytes, bar, pol);
+                    tma_load_3d(st + 2 * p.kv_bytes, &tm_q, 0, (int32_t)(p.Qw * g), 0, bar, pol);
                 }
             }
             __syncwarp();
@@ -195,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sl2 = p.scale_log2;
         const int gq = lane >> 2;       // fragment row group (query)
         const int tq = lane & 3;        // thread in group
-        uint8_t *ost = smem + p.ostage_off + warp * p.Qw * 128;
+        uint8_t *ost = smem + p.ostage_off + warp * p.Qw * kOStride;
         for (int n = 0;; ++n) {
             const long long g = blockIdx.x + (long long)n * gridDim.x;
             int f0, L, seq;
@@ -215,12 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < 2 * KT; ++j)
                     sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
                 const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;   // row this lane addresses in ldmatrix
-                const int aq = arow % p.Qw;
-                const uint32_t qrow = qbase + (uint32_t)((aq * H + h) * 128);
+                const int qline = h * p.Qw + arow % p.Qw;               // its 128-byte line in the Q tile
+                const uint32_t qrow = qbase + (uint32_t)(qline * 128);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     uint32_t a[4];
-                    ldsm_x4(qrow + (2 * ks + (lane >> 4)) * 16, a[0], a[1], a[2], a[3]);
+                    ldsm_x4(qrow + (((2 * ks + (lane >> 4)) ^ (qline & 7)) << 4), a[0], a[1], a[2], a[3]);
 #pragma unroll
                     for (int kt = 0; kt < KT; ++kt) {
                         // matrices: (keys 0-7, dims lo), (keys 0-7, dims hi),
@@ -228,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int krow = (lane & 7) + (lane >> 4) * 8;
                         const int kchunk = 2 * ks + ((lane >> 3) & 1);
                         uint32_t b0, b1, b2, b3;
-                        ldsm_x4(kbase + (h * KT + kt) * kTileBytes + swz(krow, kchunk), b0, b1, b2, b3);
+                        ldsm_x4(kbase + (kt * H + h) * kTileBytes + swz(krow, kchunk), b0, b1, b2, b3);
                         mma_16816(sacc[2 * kt], a, b0, b1);
                         mma_16816(sacc[2 * kt + 1], a, b2, b3);
                     }
@@ -277,19 +263,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l0 += __shfl_xor_sync(kFull, l0, 2);
                 l1 += __shfl_xor_sync(kFull, l1, 1);
                 l1 += __shfl_xor_sync(kFull, l1, 2);
-                // ---- a partial window: value rows L..W-1 hold frames of the
-                // next window (or utterance); zero them so nothing outside
-                // the window reaches PV
-                const int zr_end = KT == 1 ? p.W : 16 * KT;   // rows a TMA box may have filled
-                if (L < zr_end) {
-                    for (int i = lane; i < (zr_end - L) * 8; i += 32) {
-                        const int r = L + i / 8, c = i % 8;
-                        const int kt = r >> 4;
-                        *reinterpret_cast<uint4 *>(st + p.kv_bytes + (h * KT + kt) * kTileBytes + swz(r & 15, c)) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    __syncwarp();
+                // ---- value rows L..16*KT-1 hold frames past the window (the
+                // next window's, or another utterance's); zero them so
+                // nothing outside the window reaches PV (P is 0 there, but
+                // 0 * Inf would be NaN)
+                for (int i = lane; i < (16 * KT - L) * 8; i += 32) {
+                    const int r = L + i / 8, c = i % 8;
+                    const int kt = r >> 4;
+                    *reinterpret_cast<uint4 *>(st + p.kv_bytes + (kt * H + h) * kTileBytes + swz(r & 15, c)) =
+                        make_uint4(0, 0, 0, 0);
                 }
+                __syncwarp();
                 // ---- O = P V: B = values via transposing ldmatrix
                 float oacc[8][4];
 #pragma unroll
@@ -304,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int vrow = (lane & 7) + ((lane >> 3) & 1) * 8;
                         const int vchunk = 2 * jp + (lane >> 4);
                         uint32_t b0, b1, b2, b3;
-                        ldsm_x4_t(vbase + (h * KT + kt) * kTileBytes + swz(vrow, vchunk), b0, b1, b2, b3);
+                        ldsm_x4_t(vbase + (kt * H + h) * kTileBytes + swz(vrow, vchunk), b0, b1, b2, b3);
                         mma_16816(oacc[2 * jp], pa[kt], b0, b1);
                         mma_16816(oacc[2 * jp + 1], pa[kt], b2, b3);
                     }
@@ -315,19 +299,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (gq < p.Qw) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint32_t *>(ost + gq * 128 + j * 16 + tq * 4) =
+                        *reinterpret_cast<uint32_t *>(ost + gq * kOStride + j * 16 + tq * 4) =
                             pack_bf16x2(oacc[j][0] * inv0, oacc[j][1] * inv0);
                 }
                 if (gq + 8 < p.Qw) {
                     const float inv1 = 1.f / l1;
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint32_t *>(ost + (gq + 8) * 128 + j * 16 + tq * 4) =
+                        *reinterpret_cast<uint32_t *>(ost + (gq + 8) * kOStride + j * 16 + tq * 4) =
                             pack_bf16x2(oacc[j][2] * inv1, oacc[j][3] * inv1);
                 }
                 __syncwarp();
                 for (int r = 0; r < p.Qw; ++r) {
-                    const uint32_t v = *reinterpret_cast<const uint32_t *>(ost + r * 128 + lane * 4);
+                    const uint32_t v = *reinterpret_cast<const uint32_t *>(ost + r * kOStride + lane * 4);
                     *reinterpret_cast<uint32_t *>(p.out + ((long long)p.Qw * g + r) * row_elems + h * 64 + 2 * lane) = v;
                 }
                 __syncwarp();
@@ -346,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 }
 
-using WKernel = void (*)(CUtensorMap, CUtensorMap, WParams);
+using WKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, WParams);
 int g_smem_set[3][64] = {};
 
 } // namespace
@@ -385,14 +369,13 @@ extern "C" int nle_window_xattn_fwd_ex(const void *q, const void *k, const void 
     p.n_qrows = n_query_rows;
     p.heads = heads;
     p.W = window_frames;
-    p.box_rows = window_frames < 16 ? window_frames : 16;
     p.Qw = queries_per_window;
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.kv_bytes = (uint32_t)heads * KT * kTileBytes;
     p.q_bytes = (uint32_t)queries_per_window * heads * 128u;
     p.stage_bytes = (2 * p.kv_bytes + p.q_bytes + 1023) / 1024 * 1024;
-    const size_t ostage = (size_t)kComputeWarps * queries_per_window * 128;
+    const size_t ostage = (size_t)kComputeWarps * queries_per_window * kOStride;
     const size_t fixed = ostage + ((sizeof(WBars) + 127) / 128) * 128 + 1024;
     if ((size_t)di.smem_optin < fixed + 2 * (size_t)p.stage_bytes)
         return NLE_ERR_UNSUPPORTED;
@@ -409,12 +392,17 @@ extern "C" int nle_window_xattn_fwd_ex(const void *q, const void *k, const void 
     p.wait_ns = wait_limit_ns > 0 ? (unsigned long long)wait_limit_ns : 1000000000ull;
     p.flags = flags;
 
-    // K/V tensor maps: [total_frames][heads*64] bf16, boxes of 64 x min(16, W)
-    // rows (one 16-key group), 128-byte swizzle, zero fill past the end
-    CUtensorMap tk, tv;
-    const uint64_t cols = (uint64_t)heads * 64, rows = (uint64_t)total_frames;
-    if (!nle::encode_tmap_bf16_2d(&tk, k, cols, rows, cols, 64, (uint32_t)p.box_rows) ||
-        !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, cols, 64, (uint32_t)p.box_rows))
+    // Tensor maps over [rows][heads][64] bf16 as (d, row, head): K/V boxes of
+    // 16 frames x all heads, Q boxes of Qw rows x all heads; 128-byte
+    // swizzle, zero fill past the end.  (A query tensor too short for some
+    // window is reported by the kernel, which then loads no query rows for
+    // that window.)
+    CUtensorMap tk, tv, tq;
+    const uint64_t hd = (uint64_t)heads;
+    const uint64_t qrows = n_query_rows > 0 ? (uint64_t)n_query_rows : 1;
+    if (!nle::encode_tmap_bf16_heads(&tk, k, (uint64_t)total_frames, hd, hd * 64, 16, (uint32_t)heads) ||
+        !nle::encode_tmap_bf16_heads(&tv, v, (uint64_t)total_frames, hd, hd * 64, 16, (uint32_t)heads) ||
+        !nle::encode_tmap_bf16_heads(&tq, q, qrows, hd, hd * 64, (uint32_t)queries_per_window, (uint32_t)heads))
         return NLE_ERR_CUDA;
 
     WKernel kern = KT == 1 ? window_xattn_kernel<1> : window_xattn_kernel<2>;
@@ -427,7 +415,7 @@ extern "C" int nle_window_xattn_fwd_ex(const void *q, const void *k, const void 
     }
     const long long max_windows = (long long)n_seq + total_frames / window_frames;
     const int grid = (int)(max_windows < di.sm_count ? max_windows : di.sm_count);
-    kern<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tk, tv, p);
+    kern<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tk, tv, tq, p);
     return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
 }
 

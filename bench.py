@@ -341,22 +341,21 @@ def run_nle(args, rank, world, local):
     elapsed_ms = max_over_ranks(elapsed_ms, world)
     ms_step = elapsed_ms / K
 
-    # ---- end to end through the public API: host (pinned) -> device, both
-    # kernels, device -> host of both outputs, every step
-    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
-    hqw, hkw, hvw = (y[n].pin_memory() for n in ("q", "k", "v"))
-    hcu = torch.from_numpy(x["cu"]).pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    how = torch.empty(ow.shape, dtype=ow.dtype, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hqw, hkw, hvw, hcu))
-    d2h = hout.numel() * hout.element_size() + how.numel() * how.element_size()
+    # ---- end to end through the public API with HOST buffers: one
+    # nle_path_fwd_host call per step copies the step's inputs from pinned
+    # host memory, runs both kernels and copies both outputs back (chunks of
+    # utterances pipelined over two streams inside the library)
+    host = {"q": x["q"].pin_memory(), "k": x["k"].pin_memory(), "v": x["v"].pin_memory(),
+            "qw": y["q"].pin_memory(), "kw": y["k"].pin_memory(), "vw": y["v"].pin_memory(),
+            "cu": torch.from_numpy(np.ascontiguousarray(x["cu"])).pin_memory()}
+    host["out"] = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    host["out_w"] = torch.empty(ow.shape, dtype=ow.dtype, pin_memory=True)
+    devb = {"q": q, "k": k, "v": v, "qw": qw, "kw": kw, "vw": vw, "out": out, "out_w": ow, "cu": cu}
+    h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v", "qw", "kw", "vw", "cu"))
+    d2h = sum(host[n].numel() * host[n].element_size() for n in ("out", "out_w"))
 
     def e2e_step():
-        for d_, h_ in ((q, hq), (k, hk), (v, hv), (qw, hqw), (kw, hkw), (vw, hvw), (cu, hcu)):
-            d_.copy_(h_, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
-        how.copy_(ow, non_blocking=True)
+        nle.nle_path_fwd_host(host, devb, block_frames=B, window_frames=W, queries_per_window=QW, stream=sp)
 
     ke = max(3, min(K, 20))
     for _ in range(3):

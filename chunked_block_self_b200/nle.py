@@ -35,8 +35,16 @@ _i64 = ctypes.c_int64
 _f32 = ctypes.c_float
 _i32p = ctypes.POINTER(ctypes.c_int32)
 
+class PathBuffers(ctypes.Structure):
+    """nle_path_buffers: host tensors, then their device copies."""
+    _fields_ = [(n, _vp) for n in ("q", "k", "v", "out", "qw", "kw", "vw", "out_w", "cu",
+                                    "d_q", "d_k", "d_v", "d_out", "d_qw", "d_kw", "d_vw", "d_out_w", "d_cu")]
+
+
 _SIGS = {
     "nle_version": ([], _int),
+    "nle_path_fwd_host": ([ctypes.POINTER(PathBuffers), _int, _i64, _i64, _int, _int, _int, _int, _int, _int,
+                           _vp], _int),
     "nle_status_string": ([_int], ctypes.c_char_p),
     "nle_block_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int, _vp], _int),
     "nle_block_attn_fwd_ex": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int, _f32, _i64, _vp,
@@ -262,3 +270,33 @@ def nle_shard_plan_host(lengths, world_size: int, block_frames: int = 200) -> np
     _check(_lib.nle_shard_plan_host(_ptr(ln), len(ln), block_frames, world_size, _ptr(bounds)),
            "nle_shard_plan_host")
     return bounds
+
+
+# ------------------------------------------------------------------ whole path from host memory
+_PATH_NAMES = ("q", "k", "v", "out", "qw", "kw", "vw", "out_w")
+
+
+def nle_path_fwd_host(host: dict, dev: dict, block_frames: int = 200, window_frames: int = 15,
+                      queries_per_window: int = 3, n_chunks: int = 0, stream=None) -> None:
+    """Both kernels from host memory (nle_path_fwd_host).  ``host`` and ``dev``
+    map q, k, v, out, qw, kw, vw, out_w to bf16 [rows, heads, 64] tensors on the
+    CPU (pinned for overlap) and on the GPU, and cu to int32 [n_seq + 1].
+    Returns once the work is queued on ``stream``."""
+    for name in _PATH_NAMES:
+        h, d = host[name], dev[name]
+        if h.device.type != "cpu" or h.dtype != torch.bfloat16 or not h.is_contiguous():
+            raise ValueError(f"host {name}: contiguous CPU bf16 tensor required")
+        _dev_tensor(d, f"dev {name}", torch.bfloat16)
+        if h.shape != d.shape:
+            raise ValueError(f"{name}: host {tuple(h.shape)} and device {tuple(d.shape)} differ")
+    hcu, dcu = host["cu"], dev["cu"]
+    if hcu.device.type != "cpu" or hcu.dtype != torch.int32 or not hcu.is_contiguous():
+        raise ValueError("host cu: contiguous CPU int32 tensor required")
+    _dev_tensor(dcu, "dev cu", torch.int32)
+    b = PathBuffers(*[host[n].data_ptr() for n in _PATH_NAMES], hcu.data_ptr(),
+                    *[dev[n].data_ptr() for n in _PATH_NAMES], dcu.data_ptr())
+    heads = host["q"].shape[1]
+    _check(_lib.nle_path_fwd_host(ctypes.byref(b), hcu.numel() - 1, host["q"].shape[0], host["qw"].shape[0],
+                                  heads, host["q"].shape[2], block_frames, window_frames, queries_per_window,
+                                  n_chunks, _stream(stream)),
+           "nle_path_fwd_host")

@@ -30,8 +30,10 @@
  *  - q, k, v, out hold bf16 values, row-major [rows][heads][d_head]: one row
  *    per frame (or per query), heads next, d_head contiguous.  d_head must be
  *    64.  Base pointers must be 16-byte aligned.
- *  - cu_seqlens is int32 [n_seq + 1], cu[0] = 0, non-decreasing, cu[n_seq] =
- *    total_frames.  The kernels read it on the device; a sequence whose
+ *  - cu_seqlens is int32 [n_seq + 1], non-decreasing, within
+ *    [0, total_frames]; normally cu[0] = 0 and cu[n_seq] = total_frames, but
+ *    a slice of a longer cu (absolute offsets) processes just those
+ *    utterances.  The kernels read it on the device; a sequence whose
  *    offsets fall outside [0, total_frames] or decrease is skipped (no output
  *    is written for it) and, where a dev_status word is given, reported as
  *    NLE_ERR_INVALID_ARG.  No access ever leaves the buffers described by
@@ -87,7 +89,7 @@ const char *nle_status_string(int status);
  * q, k, v, out   device bf16 [total_frames][heads][64]
  * cu_seqlens     device int32 [n_seq + 1]
  * n_seq          number of packed utterances (>= 0)
- * total_frames   rows of q/k/v/out; must equal cu[n_seq]; < 2^31
+ * total_frames   rows of q/k/v/out (>= cu[n_seq]); < 2^31
  * heads          >= 1
  * d_head         must be 64
  * block_frames   frames per block, 1..256 (200 for 4 s at 50 Hz)
@@ -144,6 +146,46 @@ int nle_window_xattn_fwd_ex(const void *q, const void *k, const void *v,
                             int queries_per_window, float softmax_scale,
                             int32_t *dev_status, int flags,
                             int64_t wait_limit_ns, void *stream);
+
+/* ---------------------------------------------------------------------
+ * The whole path from host memory: block self-attention of (q, k, v) and
+ * windowed cross-attention of (qw, kw, vw) over the same n_seq packed
+ * utterances (cu), with the copies in and out.
+ *
+ * Host buffers (pinned memory lets the copies overlap the kernels):
+ *   q, k, v, out        [total_frames][heads][64] bf16
+ *   qw, out_w           [n_query_rows][heads][64] bf16, n_query_rows =
+ *                       queries_per_window * (number of windows)
+ *   kw, vw              [total_frames][heads][64] bf16
+ *   cu                  int32 [n_seq + 1], non-decreasing from 0
+ * Device buffers, owned by the caller, of the same shapes: d_q ... d_cu.
+ *
+ * The utterances are split into n_chunks chunks of consecutive utterances
+ * (0 selects 8; at most n_seq).  For each chunk the input rows are copied to
+ * the device, both kernels run on the chunk (each kernel call takes the
+ * chunk's slice of cu, whose offsets stay absolute), and the output rows are
+ * copied back; chunks alternate between two internal streams, so the copies
+ * of one chunk overlap the kernels and copies of another.  Everything is
+ * ordered after the work already on `stream`, and `stream` waits for all of
+ * it: the call returns at once, like cudaMemcpyAsync, and the host buffers
+ * must stay valid until `stream` has reached this point.
+ * Returns NLE_OK or the first error (argument checks as for the two kernel
+ * entry points; NLE_ERR_INVALID_ARG if cu is not non-decreasing from 0 or
+ * the query rows do not match the windows).
+ */
+typedef struct {
+    const void *q, *k, *v;     /* host inputs of block self-attention       */
+    void *out;                 /* host output of block self-attention       */
+    const void *qw, *kw, *vw;  /* host inputs of windowed cross-attention   */
+    void *out_w;               /* host output of windowed cross-attention   */
+    const int32_t *cu;         /* host cu_seqlens                           */
+    void *d_q, *d_k, *d_v, *d_out, *d_qw, *d_kw, *d_vw, *d_out_w;
+    int32_t *d_cu;             /* device copies (caller-owned)              */
+} nle_path_buffers;
+
+int nle_path_fwd_host(const nle_path_buffers *b, int n_seq, int64_t total_frames, int64_t n_query_rows,
+                      int heads, int d_head, int block_frames, int window_frames, int queries_per_window,
+                      int n_chunks, void *stream);
 
 /* ---------------------------------------------------------------------
  * Block / window plans (the integer scheduling the kernels perform).

@@ -255,3 +255,22 @@ def test_running_max_rescale(B, lengths, cuda_device):
     x["k"] = k.to(torch.bfloat16)
     out = _run(x, cuda_device, B=B)
     _compare(out, oracle.block_attn(x["q"], x["k"], x["v"], x["cu"], block_frames=B))
+
+
+def test_concurrent_launches_on_two_streams(cuda_device):
+    """Two launches running at once on different streams (and a third
+    queued behind one of them) must each compute every item exactly once."""
+    nle = _nle()
+    xs = [wl.block_inputs(lengths=wl.draw_lengths(4)[i * 20:(i + 1) * 20], heads=16, seed=70 + i)
+          for i in range(3)]
+    dev = [{n: x[n].to(cuda_device) for n in ("q", "k", "v")} for x in xs]
+    cus = [torch.from_numpy(x["cu"]).to(cuda_device) for x in xs]
+    outs = [torch.full_like(d["q"], float("nan")) for d in dev]
+    streams = [torch.cuda.Stream(device=cuda_device) for _ in range(2)]
+    torch.cuda.synchronize()
+    for i, st in ((0, streams[0]), (1, streams[1]), (2, streams[0])):
+        with torch.cuda.stream(st):
+            nle.nle_block_attn_fwd(dev[i]["q"], dev[i]["k"], dev[i]["v"], outs[i], cus[i], block_frames=200)
+    torch.cuda.synchronize()
+    for x, out in zip(xs, outs):
+        _compare(out, oracle.block_attn(x["q"], x["k"], x["v"], x["cu"], block_frames=200))

@@ -407,7 +407,7 @@ def run_nle(args, rank, world, local):
         "clocks": clocks.summary(),
         "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke},
-        "gpu_launches": 2 * K,
+        "gpu_launches": 2 * K * world,   # block + window kernel per step, all ranks
         "cpu_baseline": cpu_base,
     }
     if rank == 0:

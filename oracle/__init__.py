@@ -243,3 +243,6 @@ def window_xattn_rows(q, k, v, cu, qrows, heads_sel, window_frames: int = 15,
 def threads_used(n_threads: int = 0) -> int:
     """How many threads a call with ``n_threads`` uses (0 = all online cores)."""
     return n_threads if n_threads > 0 else (os.cpu_count() or 1)
+
+
+from .ctc import collapse as ctc_collapse, ctc_greedy, frame_classes as ctc_frame_classes  # noqa: E402,F401

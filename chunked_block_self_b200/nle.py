@@ -57,6 +57,7 @@ _SIGS = {
     "nle_window_plan_host": ([_vp, _int, _int, _int, _vp, _vp, _vp, _vp, _vp, _int, ctypes.POINTER(_int)],
                              _int),
     "nle_shard_plan_host": ([_vp, _int, _int, _int, _vp], _int),
+    "nle_ctc_greedy_fwd": ([_vp, _i64, _int, _vp, _int, _i64, _vp, _vp, _vp, _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -300,3 +301,31 @@ def nle_path_fwd_host(host: dict, dev: dict, block_frames: int = 200, window_fra
                                   heads, host["q"].shape[2], block_frames, window_frames, queries_per_window,
                                   n_chunks, _stream(stream)),
            "nle_path_fwd_host")
+
+
+# ------------------------------------------------------------------ CTC greedy decoding
+def nle_ctc_greedy_fwd(logits, cu_seqlens, frame_class, tokens, n_tokens, n_classes: int | None = None,
+                       stream=None) -> None:
+    """logits: CUDA bf16 [frames, row_stride] (the first n_classes used);
+    frame_class, tokens: int32 [frames]; n_tokens: int32 [n_seq]."""
+    _dev_tensor(logits, "logits", torch.bfloat16)
+    if logits.dim() != 2 or logits.stride(1) != 1:
+        raise ValueError("logits: [frames, classes] with unit stride along classes")
+    for t, n in ((cu_seqlens, "cu_seqlens"), (frame_class, "frame_class"), (tokens, "tokens"),
+                 (n_tokens, "n_tokens")):
+        _dev_tensor(t, n, torch.int32)
+    n_classes = logits.shape[1] if n_classes is None else n_classes
+    _check(_lib.nle_ctc_greedy_fwd(_ptr(logits), logits.stride(0), n_classes, _ptr(cu_seqlens),
+                                   cu_seqlens.numel() - 1, logits.shape[0], _ptr(frame_class), _ptr(tokens),
+                                   _ptr(n_tokens), _stream(stream)),
+           "nle_ctc_greedy_fwd")
+
+
+def ctc_greedy(logits, cu_seqlens, n_classes: int | None = None, stream=None):
+    """(frame_class, tokens, n_tokens) of CTC greedy decoding on the GPU."""
+    frames, n_seq = logits.shape[0], cu_seqlens.numel() - 1
+    frame_class = torch.empty(frames, dtype=torch.int32, device=logits.device)
+    tokens = torch.full((frames,), -1, dtype=torch.int32, device=logits.device)
+    n_tokens = torch.empty(n_seq, dtype=torch.int32, device=logits.device)
+    nle_ctc_greedy_fwd(logits, cu_seqlens, frame_class, tokens, n_tokens, n_classes, stream)
+    return frame_class, tokens, n_tokens

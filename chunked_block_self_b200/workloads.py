@@ -151,3 +151,53 @@ def window_inputs(n_query_rows: int, cfg: int | None = 5, seed: int | None = Non
     q = bf16_normal(rng, (int(n_query_rows), heads, d_head), factor)
     return dict(q=q, k=k, v=v, cu=cu, lengths=lengths, heads=heads, d_head=d_head,
                 total=total)
+
+
+# ------------------------------------------------------------------ CTC head logits
+CTC_CLASSES = 100353   # vocab + 1, blank at class 0 (q4-RTN ONNX page, decode note)
+
+
+def ctc_logits(lengths, n_classes: int = CTC_CLASSES, seed: int = 2000, row_stride: int | None = None,
+               device=None) -> torch.Tensor:
+    """bf16 [frames, row_stride] logits shaped like a CTC head's output (only
+    the first n_classes of a row are meaningful; padding is random too):
+    N(0, 1) everywhere, then frames are drawn in runs of 1-4 -- about 60 %
+    of the runs boost the blank (class 0) by 6, the rest boost one random
+    class by 6 -- so that blanks, repeated classes and separated repeats all
+    occur.  A few frames get an exact tie between two boosted classes.
+    With device=None the values come from numpy's default_rng(seed) on the
+    host; with a CUDA device, from a seeded torch generator on the device
+    (other values, same structure)."""
+    frames = int(np.sum(lengths))
+    stride = n_classes if row_stride is None else row_stride
+    if device is None:
+        rng = np.random.default_rng(seed)
+        x = torch.from_numpy(rng.standard_normal((frames, stride), dtype=np.float32))
+        # runs of boosted classes
+        cls = np.empty(frames, np.int64)
+        i = 0
+        while i < frames:
+            run = int(rng.integers(1, 5))
+            c = 0 if rng.random() < 0.6 else int(rng.integers(1, n_classes))
+            cls[i:i + run] = c
+            i += run
+        ties = rng.random(frames) < 0.02
+        tie_cls = rng.integers(0, n_classes, frames)
+        x[np.arange(frames), cls] = 6.0
+        x[np.nonzero(ties)[0], tie_cls[ties]] = 6.0
+        return x.to(torch.bfloat16)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    x = torch.randn((frames, stride), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    runs = torch.randint(1, 5, (frames,), generator=g, device=device)
+    starts = torch.cumsum(runs, 0) - runs
+    starts = starts[starts < frames]
+    run_id = torch.zeros(frames, dtype=torch.int64, device=device)
+    run_id[starts[1:]] = 1
+    run_id = torch.cumsum(run_id, 0)
+    n_runs = int(starts.numel())
+    blank = torch.rand((n_runs,), generator=g, device=device) < 0.6
+    rcls = torch.where(blank, torch.zeros((), dtype=torch.int64, device=device),
+                       torch.randint(1, n_classes, (n_runs,), generator=g, device=device))
+    x[torch.arange(frames, device=device), rcls[run_id]] = 6.0
+    return x

@@ -148,6 +148,32 @@ int nle_window_xattn_fwd_ex(const void *q, const void *k, const void *v,
                             int64_t wait_limit_ns, void *stream);
 
 /* ---------------------------------------------------------------------
+ * CTC greedy decoding of the encoder's CTC head (q4-RTN ONNX page,
+ * "Inference note (NAR decode)"): the head emits n_classes per frame with
+ * the blank at class 0, and a non-blank class c is token c - 1.  Per frame
+ * the class of the largest logit is taken (bf16 compared exactly; among
+ * equal largest logits the lowest class; NaN logits never win); per
+ * utterance, runs of equal consecutive classes become one (runs never cross
+ * utterances), blanks are dropped and classes become tokens.
+ *
+ * logits       device bf16 [total_frames][row_stride]; the first n_classes
+ *              of each row are used; base 16-byte aligned, rows may start
+ *              at any element
+ * row_stride   elements between frames, >= n_classes
+ * cu_seqlens   device int32 [n_seq + 1] (as for the attention kernels)
+ * frame_class  device int32 [total_frames], out: class of each frame
+ * tokens       device int32 [total_frames], out: utterance i's tokens at
+ *              tokens[cu[i]] .. tokens[cu[i] + n_tokens[i] - 1]; the rest of
+ *              its frame range is left untouched
+ * n_tokens     device int32 [n_seq], out: tokens of each utterance (0 for an
+ *              utterance whose offsets are invalid)
+ * Two kernels on `stream` (argmax, then collapse); no allocation.
+ */
+int nle_ctc_greedy_fwd(const void *logits, int64_t row_stride, int n_classes, const int32_t *cu_seqlens,
+                       int n_seq, int64_t total_frames, int32_t *frame_class, int32_t *tokens,
+                       int32_t *n_tokens, void *stream);
+
+/* ---------------------------------------------------------------------
  * The whole path from host memory: block self-attention of (q, k, v) and
  * windowed cross-attention of (qw, kw, vw) over the same n_seq packed
  * utterances (cu), with the copies in and out.

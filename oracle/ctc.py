@@ -7,6 +7,8 @@ of the largest logit, collapses runs of equal consecutive classes into one,
 drops the blank, and subtracts 1.  Readings taken where the page is silent:
 - the logits are bf16 (the model card's inference is bf16) and are compared
   exactly; among equal largest logits the lowest class wins;
+- a NaN logit is no candidate (it carries no ordering); a frame whose logits
+  are all NaN takes the blank;
 - runs are collapsed within one utterance of the packed batch only;
 - a blank frame between two equal classes separates them (both are kept).
 
@@ -33,10 +35,16 @@ def _as_f64(logits) -> np.ndarray:
 
 
 def frame_classes(logits) -> np.ndarray:
-    """Class of the largest logit of each frame ([T, C] -> [T] int64); the
-    first (lowest) class among equal maxima."""
+    """Class of the largest logit of each frame ([T, C] -> [T] int64): the
+    first (lowest) class among equal maxima, NaN logits skipped, the blank
+    when a frame has no other candidate."""
     x = _as_f64(logits)
-    return np.argmax(x, axis=1).astype(np.int64)
+    out = np.zeros(x.shape[0], np.int64)
+    for t in range(x.shape[0]):
+        ok = np.nonzero(~np.isnan(x[t]))[0]   # the candidate classes, ascending
+        if ok.size:
+            out[t] = ok[np.argmax(x[t, ok])]   # first (lowest) of the maxima
+    return out
 
 
 def collapse(classes, cu, blank: int = 0) -> list[list[int]]:

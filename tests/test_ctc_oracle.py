@@ -76,3 +76,24 @@ def test_planted_mistake_is_caught():
     wrong = oracle.ctc_collapse(cls, [0, len(cls)])      # boundary ignored
     flat = [t for u in case["tokens"] for t in u]
     assert wrong[0] != flat
+
+
+# Non-finite and signed-zero logits, worked by hand.  Reading taken where the
+# page is silent: a NaN logit is no candidate; a frame of NaNs only takes the
+# blank; -0 and +0 are equal (the lower class wins); infinities order as usual.
+NONFINITE = [
+    ([np.nan, 1.0, 1.0], 1),
+    ([np.nan, np.nan, np.nan], 0),
+    ([np.nan, -np.inf, -np.inf], 1),
+    ([-np.inf, np.nan], 0),
+    ([-np.inf, -np.inf, -np.inf], 0),
+    ([2.0, np.inf, np.nan, np.inf], 1),
+    ([-0.0, 0.0, -1.0], 0),
+    ([-1.0, 0.0, -0.0], 1),
+    ([np.nan, -3.0, np.nan, -2.0, np.nan], 3),
+]
+
+
+@pytest.mark.parametrize("row,cls", NONFINITE)
+def test_nonfinite_and_signed_zero(row, cls):
+    assert oracle.ctc_frame_classes(_bf16_bits([row])).tolist() == [cls]

@@ -240,6 +240,25 @@ def window_xattn_rows(q, k, v, cu, qrows, heads_sel, window_frames: int = 15,
     return out
 
 
+def _one_block(cu) -> int:
+    """A block length that holds every utterance of cu whole."""
+    cu = np.asarray(cu, np.int64)
+    return max(1, int(np.max(np.diff(cu)))) if len(cu) > 1 else 1
+
+
+def varlen_attn(q, k, v, cu, scale: float | None = None, n_threads: int = 0) -> np.ndarray:
+    """Full bidirectional attention inside each packed utterance (no blocks;
+    the editor's attention with the causal mask removed, granite-speech-
+    4.1-2b-nar model card, "Model Architecture" (3)): the block definition
+    with one block per utterance, float64 [total_frames, heads, d]."""
+    return block_attn(q, k, v, cu, block_frames=_one_block(cu), scale=scale, n_threads=n_threads)
+
+
+def varlen_attn_rows(q, k, v, cu, rows, heads_sel, scale: float | None = None) -> np.ndarray:
+    """Full-utterance attention outputs at selected (frame, head) pairs."""
+    return block_attn_rows(q, k, v, cu, rows, heads_sel, block_frames=_one_block(cu), scale=scale)
+
+
 def threads_used(n_threads: int = 0) -> int:
     """How many threads a call with ``n_threads`` uses (0 = all online cores)."""
     return n_threads if n_threads > 0 else (os.cpu_count() or 1)

@@ -383,7 +383,75 @@ def run_nle(args, rank, world, local):
                               f"({fr} frames; block + window oracle, {t:.1f} s, fp64, {threads} threads), "
                               f"{cpu_info()}"}
 
+    # ---- downstream of the encoder, on the same utterances: the BPE head's
+    # posterior-weighted pooling (windows of 2 frames, weights from a
+    # 256-class mid-layer head) and CTC greedy decoding of the BPE head's
+    # logits (100,353 classes, one row per pooled window); inputs generated
+    # on the device, L2 flushed before every timed launch
+    pool = ctc = None
+    if not args.no_ctc:
+        del host, devb
+        torch.cuda.empty_cache()
+        clen = lengths if args.ctc_utts <= 0 else lengths[:args.ctc_utts]
+        cu_f = torch.from_numpy(wl.cu_seqlens(clen)).to(dev)
+        rows_u = [-(-int(t) // wl.POOL_FRAMES) for t in clen]
+        cu_r = torch.from_numpy(wl.cu_seqlens(rows_u)).to(dev)
+        n_rows, n_fr = int(sum(rows_u)), int(sum(int(t) for t in clen))
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+        def timed(fn, reps):
+            ts = []
+            for _ in range(reps):
+                flush.fill_(1)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            return float(np.mean(ts))
+
+        px = wl.pool_inputs(clen, seed=wl.default_seed(CFG) + 4000 + rank, device=dev)
+        pooled = torch.empty((n_rows, wl.HIDDEN_DIM), dtype=torch.bfloat16, device=dev)
+        pw = torch.empty(n_fr, dtype=torch.float32, device=dev)
+
+        def pool_step():
+            nle.nle_posterior_pool_fwd(px["hidden"], px["logits"], cu_f, pooled, pw, wl.POOL_FRAMES, stream=sp)
+
+        for _ in range(3):
+            pool_step()
+        pool_ms = timed(pool_step, 20)
+        # hidden and logits once, pooled rows and weights written
+        pool_bytes = n_fr * (wl.HIDDEN_DIM + wl.CHAR_CLASSES) * 2 + n_rows * wl.HIDDEN_DIM * 2 + n_fr * 4
+        pool = {"frames": n_fr, "rows": n_rows, "pool_frames": wl.POOL_FRAMES, "dim": wl.HIDDEN_DIM,
+                "char_classes": wl.CHAR_CLASSES, "ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
+                "algorithmic_bytes": pool_bytes, "l2": "flushed (256 MB write) before each launch", "kernels": 1}
+        del px, pooled, pw
+
+        logits = wl.ctc_logits(rows_u, seed=wl.default_seed(CFG) + 3000 + rank, device=dev)
+        fcl = torch.empty(n_rows, dtype=torch.int32, device=dev)
+        tok = torch.empty_like(fcl)
+        ntk = torch.empty(len(clen), dtype=torch.int32, device=dev)
+
+        def ctc_step():
+            nle.nle_ctc_greedy_fwd(logits, cu_r, fcl, tok, ntk, stream=sp)
+
+        for _ in range(3):
+            ctc_step()
+        ctc_ms = timed(ctc_step, 10)
+        # logits once; frame classes written, read twice by the collapse;
+        # tokens written; one count per utterance
+        ctc_bytes = logits.numel() * 2 + n_rows * 12 + len(clen) * 4
+        ctc = {"rows": n_rows, "utterances": len(clen), "classes": int(logits.shape[1]), "ms": ctc_ms,
+               "rows_per_s": n_rows / (ctc_ms * 1e-3), "gbs": ctc_bytes / (ctc_ms * 1e-3) / 1e9,
+               "algorithmic_bytes": ctc_bytes, "l2": "flushed (256 MB write) before each launch", "kernels": 2}
+        del logits, flush
+        torch.cuda.empty_cache()
+
     hbm_peak, tf_peak, tf_sust, peak_src = measured_peaks()
+    for extra in (pool, ctc):
+        if extra is not None:
+            extra["pct_of_hbm_peak"] = 100.0 * extra["gbs"] / hbm_peak
     achieved_gbs = by_blk / (t_blk * 1e-3) / 1e9
     traffic = ncu_traffic("block_attn", by_blk)
     blk_tflops = f_blk / (t_blk * 1e-3) / 1e12
@@ -407,6 +475,8 @@ def run_nle(args, rank, world, local):
         "clocks": clocks.summary(),
         "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke},
+        "posterior_pool": pool,
+        "ctc_decode": ctc,
         "gpu_launches": 2 * K * world,   # block + window kernel per step, all ranks
         "cpu_baseline": cpu_base,
     }
@@ -423,6 +493,10 @@ def main():
     ap.add_argument("--impl", choices=["nle", "reference"], default="nle")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget (N=1 only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ctc", action="store_true",
+                    help="skip the pooling and CTC decoding measurements")
+    ap.add_argument("--ctc-utts", type=int, default=0,
+                    help="pool and decode only the first N utterances (0: the whole batch)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -10,10 +10,11 @@
 //   ctc_argmax_kernel    streams the logits once (HBM-bound: 2 bytes per
 //                        class per frame).  A CTA takes whole frames; its
 //                        threads read the frame's row as 16-byte aligned
-//                        chunks (rows may start at any 2-byte offset: the
-//                        chunk elements outside the row are masked), keep
+//                        chunks (rows may start at any 2-byte offset), keep
 //                        the largest value and its lowest class, and reduce
-//                        across the CTA (ties go to the lowest class).
+//                        across the CTA (ties go to the lowest class; NaN
+//                        logits are skipped; a frame of NaNs takes the
+//                        blank).
 //   ctc_collapse_kernel  one CTA per utterance: keeps frame i when its class
 //                        is not the blank and differs from frame i - 1's
 //                        (the utterance's first frame has no predecessor),
@@ -21,6 +22,7 @@
 //                        scan at the utterance's own frame offset, and
 //                        writes the count.
 #include <climits>
+#include <cstring>
 
 #include "nle.h"
 #include "nle_device.cuh"
@@ -39,6 +41,38 @@ __device__ __forceinline__ bool better(float v, int c, float bv, int bc)
     return v > bv || (v == bv && c < bc);
 }
 
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t w)
+{
+    __nv_bfloat162 r;
+    memcpy(&r, &w, 4);
+    return r;
+}
+
+// largest of a chunk's 8 values (NaN only when all 8 are NaN)
+__device__ __forceinline__ float chunk_max(const uint4 &q)
+{
+    const __nv_bfloat162 m =
+        __hmax2(__hmax2(as_bf162(q.x), as_bf162(q.y)), __hmax2(as_bf162(q.z), as_bf162(q.w)));
+    uint32_t u;
+    memcpy(&u, &m, 4);
+    return fmaxf(bf16_lo(u), bf16_hi(u));
+}
+
+__device__ __forceinline__ float chunk_elem(const uint4 &q, int e)
+{
+    const uint32_t w = e < 2 ? q.x : e < 4 ? q.y : e < 6 ? q.z : q.w;
+    return e & 1 ? bf16_hi(w) : bf16_lo(w);
+}
+
+// Per frame: a CTA reads the row's whole 16-byte chunks with 16-byte loads
+// and keeps, per thread, only the largest chunk maximum and the first chunk
+// that reached it (packed bf16 max: about one instruction per logit, so the
+// loop stays under the HBM time); the class inside that chunk is found by
+// reading the chunk once more.  The row's elements before its first 16-byte
+// boundary and after its last one (at most 7 each) are read one by one.
 __global__ void __launch_bounds__(kArgmaxThreads)
     ctc_argmax_kernel(const __nv_bfloat16 *__restrict__ logits, long long row_stride, int n_classes,
                       long long total_frames, int32_t *__restrict__ frame_class)
@@ -46,66 +80,79 @@ __global__ void __launch_bounds__(kArgmaxThreads)
     __shared__ float s_val[kArgmaxThreads / 32];
     __shared__ int s_cls[kArgmaxThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // 16-byte chunks are only read below the last 16-byte boundary of the
-    // tensor; a row's elements past it (at most 7) are read one by one
-    const uintptr_t end = reinterpret_cast<uintptr_t>(logits + (total_frames - 1) * row_stride + n_classes);
-    const uintptr_t end16 = end & ~uintptr_t(15);
     for (long long r = blockIdx.x; r < total_frames; r += gridDim.x) {
-        const uintptr_t row = reinterpret_cast<uintptr_t>(logits + r * row_stride);
-        const uintptr_t a0 = row & ~uintptr_t(15);
-        const uintptr_t row_end = row + 2ull * n_classes;
-        const long long n_cover = (long long)((row_end - a0 + 15) >> 4);   // chunks covering the row
-        const long long n_safe = (long long)((end16 - a0) >> 4);             // chunks below end16
-        const long long n_chunks = n_cover < n_safe ? n_cover : n_safe;
-        const bool tail = n_cover > n_chunks;
-        // class of the first element of chunk 0 (negative: before the row)
-        const long long c_first = -(long long)((row - a0) >> 1);
-        float bv = -INFINITY;
-        int bc = INT_MAX;
-        long long k = tid;
-        // four independent 16-byte loads in flight per thread
-        for (; k + 3 * kArgmaxThreads < n_chunks; k += 4 * kArgmaxThreads) {
+        const __nv_bfloat16 *row = logits + r * row_stride;
+        // logits are 16-byte aligned, so a row starts on a 2-byte boundary
+        const int mis = (int)((reinterpret_cast<uintptr_t>(row) & 15) >> 1);
+        const int head = min((8 - mis) & 7, n_classes);   // elements before the first boundary
+        const int nfull = (n_classes - head) >> 3;        // whole chunks
+        const int tail0 = head + 8 * nfull;                // elements [tail0, n_classes) after them
+        const uint4 *chunks = reinterpret_cast<const uint4 *>(row + head);
+
+        float best = -INFINITY;
+        int bk = -1;   // first chunk of this thread whose maximum is best (-1: none above -inf)
+        int k = tid;
+        for (; k + 3 * kArgmaxThreads < nfull; k += 4 * kArgmaxThreads) {
             uint4 q[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                q[j] = __ldcs(reinterpret_cast<const uint4 *>(a0) + k + j * kArgmaxThreads);
+                q[j] = __ldcs(chunks + k + j * kArgmaxThreads);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const long long c0 = c_first + 8 * (k + j * kArgmaxThreads);
-                const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+                const float f = chunk_max(q[j]);
+                if (f > best) {
+                    best = f;
+                    bk = k + j * kArgmaxThreads;
+                }
+            }
+        }
+        for (; k < nfull; k += kArgmaxThreads) {
+            const float f = chunk_max(__ldcs(chunks + k));
+            if (f > best) {
+                best = f;
+                bk = k;
+            }
+        }
+
+        float bv = -INFINITY;
+        int bc = INT_MAX;
+        if (bk >= 0) {
+            // the lowest class of the chunk that holds the maximum
+            const uint4 q = chunks[bk];
+#pragma unroll
+            for (int e = 7; e >= 0; --e)
+                if (chunk_elem(q, e) == best)
+                    bc = head + 8 * bk + e;
+            bv = best;
+        } else {
+            // rare: this thread's chunks hold only -inf and NaN; the first
+            // -inf is its candidate
+            for (int kk = tid; kk < nfull; kk += kArgmaxThreads) {
+                const uint4 q = chunks[kk];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const long long c = c0 + e;
-                    const float v = __uint_as_float(e & 1 ? w[e >> 1] & 0xffff0000u : w[e >> 1] << 16);
-                    if (c >= 0 && c < n_classes && better(v, (int)c, bv, bc)) {
+                    const float v = chunk_elem(q, e);
+                    const int c = head + 8 * kk + e;
+                    if (better(v, c, bv, bc)) {
                         bv = v;
-                        bc = (int)c;
+                        bc = c;
                     }
                 }
             }
         }
-        if (tail && tid == 0) {
-            // the row's elements from end16 on: element loads only
-            const __nv_bfloat16 *p = reinterpret_cast<const __nv_bfloat16 *>(a0) + 8 * n_chunks;
-            for (long long c = c_first + 8 * n_chunks; c < n_classes; ++c, ++p) {
-                const float v = __bfloat162float(*p);
-                if (c >= 0 && better(v, (int)c, bv, bc)) {
+        // the row's loose elements: the head on lanes of warp 0, the tail on
+        // lanes of warp 1
+        {
+            int c = -1;
+            if (tid < head)
+                c = tid;
+            else if (tid >= 32 && tid - 32 < n_classes - tail0)
+                c = tail0 + tid - 32;
+            if (c >= 0) {
+                const float v = __bfloat162float(row[c]);
+                if (better(v, c, bv, bc)) {
                     bv = v;
-                    bc = (int)c;
-                }
-            }
-        }
-        for (; k < n_chunks; k += kArgmaxThreads) {
-            const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(a0) + k);
-            const long long c0 = c_first + 8 * k;
-            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const long long c = c0 + e;
-                const float v = __uint_as_float(e & 1 ? w[e >> 1] & 0xffff0000u : w[e >> 1] << 16);
-                if (c >= 0 && c < n_classes && better(v, (int)c, bv, bc)) {
-                    bv = v;
-                    bc = (int)c;
+                    bc = c;
                 }
             }
         }
@@ -129,7 +176,7 @@ __global__ void __launch_bounds__(kArgmaxThreads)
                     bv = s_val[i];
                     bc = s_cls[i];
                 }
-            // all logits NaN: no class compared larger; report the blank
+            // all logits NaN: no candidate; the blank
             frame_class[r] = bc == INT_MAX ? 0 : bc;
         }
         __syncthreads();

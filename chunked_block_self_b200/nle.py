@@ -58,6 +58,8 @@ _SIGS = {
                              _int),
     "nle_shard_plan_host": ([_vp, _int, _int, _int, _vp], _int),
     "nle_ctc_greedy_fwd": ([_vp, _i64, _int, _vp, _int, _i64, _vp, _vp, _vp, _vp], _int),
+    "nle_posterior_pool_fwd": ([_vp, _i64, _int, _vp, _i64, _int, _vp, _int, _i64, _int, _i64, _vp, _vp, _vp,
+                                _vp], _int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -329,3 +331,51 @@ def ctc_greedy(logits, cu_seqlens, n_classes: int | None = None, stream=None):
     n_tokens = torch.empty(n_seq, dtype=torch.int32, device=logits.device)
     nle_ctc_greedy_fwd(logits, cu_seqlens, frame_class, tokens, n_tokens, n_classes, stream)
     return frame_class, tokens, n_tokens
+
+
+# ------------------------------------------------------------------ posterior-weighted pooling
+def pooled_rows(cu_host, pool_frames: int = 2) -> int:
+    """Rows of the pooled output: one per window of pool_frames frames."""
+    return window_query_rows(cu_host, pool_frames, 1)
+
+
+def nle_posterior_pool_fwd(hidden, logits, cu_seqlens, pooled, weights=None, pool_frames: int = 2,
+                           n_classes: int | None = None, dev_status=None, stream=None) -> None:
+    """hidden: CUDA bf16 [frames, hidden_stride] (the first pooled.shape[1]
+    columns used); logits: CUDA bf16 [frames, logits_stride] of the mid-layer
+    head (the first n_classes used, blank at 0); pooled: bf16 [rows, dim];
+    weights: None or float32 [frames]; dev_status: None or int32 [1]."""
+    _dev_tensor(hidden, "hidden", torch.bfloat16)
+    _dev_tensor(logits, "logits", torch.bfloat16)
+    _dev_tensor(pooled, "pooled", torch.bfloat16)
+    _dev_tensor(cu_seqlens, "cu_seqlens", torch.int32)
+    for t, n in ((hidden, "hidden"), (logits, "logits"), (pooled, "pooled")):
+        if t.dim() != 2 or t.stride(1) != 1:
+            raise ValueError(f"{n}: 2-D with unit stride along its last dimension")
+    if not pooled.is_contiguous():
+        raise ValueError("pooled: contiguous [rows, dim] required")
+    if weights is not None:
+        _dev_tensor(weights, "weights", torch.float32)
+    if dev_status is not None:
+        _dev_tensor(dev_status, "dev_status", torch.int32)
+    if hidden.shape[0] != logits.shape[0]:
+        raise ValueError("hidden and logits: different frame counts")
+    n_classes = logits.shape[1] if n_classes is None else n_classes
+    _check(_lib.nle_posterior_pool_fwd(_ptr(hidden), hidden.stride(0), pooled.shape[1], _ptr(logits),
+                                       logits.stride(0), n_classes, _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                                       hidden.shape[0], pool_frames, pooled.shape[0], _ptr(pooled),
+                                       _ptr(weights), _ptr(dev_status), _stream(stream)),
+           "nle_posterior_pool_fwd")
+
+
+def posterior_pool(hidden, logits, cu_seqlens, pool_frames: int = 2, n_rows: int | None = None,
+                   dim: int | None = None, n_classes: int | None = None, stream=None):
+    """(pooled bf16 [rows, dim], weights float32 [frames]) on the GPU.  n_rows
+    defaults to the windows of cu_seqlens (read back to the host)."""
+    if n_rows is None:
+        n_rows = pooled_rows(cu_seqlens.cpu(), pool_frames)
+    dim = hidden.shape[1] if dim is None else dim
+    pooled = torch.empty((n_rows, dim), dtype=torch.bfloat16, device=hidden.device)
+    weights = torch.empty(hidden.shape[0], dtype=torch.float32, device=hidden.device)
+    nle_posterior_pool_fwd(hidden, logits, cu_seqlens, pooled, weights, pool_frames, n_classes, None, stream)
+    return pooled, weights

@@ -201,3 +201,60 @@ def ctc_logits(lengths, n_classes: int = CTC_CLASSES, seed: int = 2000, row_stri
                        torch.randint(1, n_classes, (n_runs,), generator=g, device=device))
     x[torch.arange(frames, device=device), rcls[run_id]] = 6.0
     return x
+
+
+# ------------------------------------------------------------------ posterior-weighted pooling
+POOL_FRAMES = 2       # a window of 4 10-ms input frames = 2 encoder frames at 50 Hz
+HIDDEN_DIM = 1024     # encoder width: 16 heads x 64
+CHAR_CLASSES = 256    # mid-layer (character) head classes: not on the pages; a stand-in
+
+
+def pool_inputs(lengths, dim: int = HIDDEN_DIM, n_classes: int = CHAR_CLASSES, seed: int = 3000,
+                hidden_stride: int | None = None, logits_stride: int | None = None, device=None) -> dict:
+    """Inputs of the posterior-weighted pooling: hidden bf16 [frames,
+    hidden_stride] (N(0, 1); the first dim columns used) and the mid-layer
+    head's logits bf16 [frames, logits_stride] (N(0, 2^2); the first
+    n_classes used).  Frames come in runs of 1-6: about half of the runs
+    boost the blank (class 0) by 2-10, so blank probabilities range from
+    near 0 to near 1; 2 % of frames get every non-blank logit -inf (weight
+    exactly 0) and 1 % get a -inf blank (weight exactly 1).  With
+    device=None the values come from numpy's default_rng(seed) on the host,
+    else from a seeded torch generator on that device (same structure)."""
+    frames = int(np.sum(lengths))
+    hs = dim if hidden_stride is None else hidden_stride
+    zs = n_classes if logits_stride is None else logits_stride
+    if device is None:
+        rng = np.random.default_rng(seed)
+        h = torch.from_numpy(rng.standard_normal((frames, hs), dtype=np.float32))
+        z = rng.standard_normal((frames, zs), dtype=np.float32) * 2.0
+        i = 0
+        while i < frames:
+            run = int(rng.integers(1, 7))
+            if rng.random() < 0.5:
+                z[i:i + run, 0] += np.float32(rng.uniform(2.0, 10.0))
+            i += run
+        if n_classes > 1:
+            dead = rng.random(frames) < 0.02
+            z[np.ix_(np.nonzero(dead)[0], np.arange(1, n_classes))] = -np.inf
+        z[rng.random(frames) < 0.01, 0] = -np.inf
+        return dict(hidden=h.to(torch.bfloat16), logits=torch.from_numpy(z).to(torch.bfloat16))
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    h = torch.randn((frames, hs), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    z = torch.randn((frames, zs), generator=g, device=device, dtype=torch.float32) * 2.0
+    runs = torch.randint(1, 7, (frames,), generator=g, device=device)
+    starts = torch.cumsum(runs, 0) - runs
+    starts = starts[starts < frames]
+    run_id = torch.zeros(frames, dtype=torch.int64, device=device)
+    run_id[starts[1:]] = 1
+    run_id = torch.cumsum(run_id, 0)
+    n_runs = int(starts.numel())
+    boost = torch.where(torch.rand((n_runs,), generator=g, device=device) < 0.5,
+                        2.0 + 8.0 * torch.rand((n_runs,), generator=g, device=device),
+                        torch.zeros((), device=device))
+    z[:, 0] += boost[run_id]
+    if n_classes > 1:
+        dead = torch.rand((frames,), generator=g, device=device) < 0.02
+        z[dead, 1:n_classes] = -float("inf")
+    z[torch.rand((frames,), generator=g, device=device) < 0.01, 0] = -float("inf")
+    return dict(hidden=h, logits=z.to(torch.bfloat16))

@@ -152,7 +152,8 @@ int nle_window_xattn_fwd_ex(const void *q, const void *k, const void *v,
  * "Inference note (NAR decode)"): the head emits n_classes per frame with
  * the blank at class 0, and a non-blank class c is token c - 1.  Per frame
  * the class of the largest logit is taken (bf16 compared exactly; among
- * equal largest logits the lowest class; NaN logits never win); per
+ * equal largest logits the lowest class, -0 equal to +0; NaN logits are no
+ * candidates and a frame of NaNs takes the blank); per
  * utterance, runs of equal consecutive classes become one (runs never cross
  * utterances), blanks are dropped and classes become tokens.
  *
@@ -168,10 +169,55 @@ int nle_window_xattn_fwd_ex(const void *q, const void *k, const void *v,
  * n_tokens     device int32 [n_seq], out: tokens of each utterance (0 for an
  *              utterance whose offsets are invalid)
  * Two kernels on `stream` (argmax, then collapse); no allocation.
+ * Errors (before launch): NLE_ERR_INVALID_ARG for n_seq < 0, total_frames
+ * < 0, n_classes < 1, row_stride < n_classes or a null pointer with work to
+ * do; NLE_ERR_UNSUPPORTED for total_frames > 2^31 - 1 or a device other than
+ * compute capability 10.x; NLE_ERR_MISALIGNED when logits is not 16-byte
+ * aligned; NLE_ERR_CUDA for a launch error.
  */
 int nle_ctc_greedy_fwd(const void *logits, int64_t row_stride, int n_classes, const int32_t *cu_seqlens,
                        int n_seq, int64_t total_frames, int32_t *frame_class, int32_t *tokens,
                        int32_t *n_tokens, void *stream);
+
+/* ---------------------------------------------------------------------
+ * Posterior-weighted pooling for the BPE CTC head (granite-speech-4.1-2b-nar
+ * model card, "Model Architecture" (1) CTC Speech Encoder): frames are
+ * pooled over windows, each weighted by 1 - blank probability of the
+ * mid-layer CTC head.  Per utterance, windows of pool_frames frames are cut
+ * from its frame 0 without overlap (the last may be partial); window g of
+ * the packed batch is pooled row g:
+ *     w_t = 1 - softmax(z_t)[0],   pooled_g = sum_t w_t h_t / sum_t w_t,
+ * a zero row when every weight of the window is 0 (w_t = 0 exactly when
+ * every non-blank logit is -inf).  The page's window of 4 counts 10 ms input
+ * frames, i.e. pool_frames = 2 encoder frames at 50 Hz (844 mel frames give
+ * 211 rows of the BPE head).  fp32 arithmetic, weights formed in the log
+ * domain; pooled rows rounded to bf16.  Logits must be finite or -inf.
+ *
+ * hidden         device bf16 [total_frames][hidden_stride]; the first dim
+ *                columns are pooled; 16-byte aligned, hidden_stride and dim
+ *                multiples of 8
+ * logits         device bf16 [total_frames][logits_stride] of the mid-layer
+ *                head, blank at class 0; the first n_classes used
+ * cu_seqlens     device int32 [n_seq + 1] (as for the attention kernels;
+ *                invalid utterances are skipped and reported)
+ * n_pooled_rows  rows of `pooled`: sum_i ceil(T_i / pool_frames); windows
+ *                past it are not written and are reported
+ * pooled         device bf16 [n_pooled_rows][dim], out; 16-byte aligned
+ * weights        nullable device float32 [total_frames], out: w_t
+ * dev_status     nullable device int32, receives NLE_ERR_INVALID_ARG for a
+ *                bad utterance or too few rows (never reset by the library)
+ * One kernel on `stream`; no allocation.  Errors (before launch):
+ * NLE_ERR_INVALID_ARG for negative sizes, dim < 1, n_classes < 1,
+ * pool_frames < 1, a stride below its width or a null pointer with work to
+ * do; NLE_ERR_MISALIGNED for dim or hidden_stride not a multiple of 8,
+ * hidden or pooled not 16-byte aligned; NLE_ERR_UNSUPPORTED for
+ * total_frames > 2^31 - 1, pool_frames > 4096 or a device other than
+ * compute capability 10.x; NLE_ERR_CUDA for a launch error.
+ */
+int nle_posterior_pool_fwd(const void *hidden, int64_t hidden_stride, int dim, const void *logits,
+                           int64_t logits_stride, int n_classes, const int32_t *cu_seqlens, int n_seq,
+                           int64_t total_frames, int pool_frames, int64_t n_pooled_rows, void *pooled,
+                           float *weights, int32_t *dev_status, void *stream);
 
 /* ---------------------------------------------------------------------
  * The whole path from host memory: block self-attention of (q, k, v) and

@@ -99,3 +99,38 @@ def test_invalid_offsets_give_zero_tokens(cuda_device):
     cls, toks = oracle.ctc_greedy(logits, [0, 10])
     assert nt[0] == len(toks[0]) and tok[:nt[0]].tolist() == toks[0]
     assert nt[1] == 0
+
+
+@pytest.mark.parametrize("n_classes,pad", [(1000, 3), (100353, 0), (13, 1)])
+def test_nonfinite_signed_zero_and_ties(n_classes, pad, cuda_device):
+    """Rows built to hit every branch of the argmax: NaN-only and -inf-only
+    rows, NaN mixed with -inf, infinities, -0 against +0, the maximum repeated
+    in several chunks, at the first and last class (the loose elements
+    before and after the row's 16-byte chunks), and rows of few distinct
+    values (ties everywhere).  NaN logits are no candidates."""
+    rng = np.random.default_rng(n_classes)
+    C = n_classes
+    rows = []
+    nan, inf = np.float32(np.nan), np.float32(np.inf)
+
+    def r(fill=None):
+        return (np.full(C, fill, np.float32) if fill is not None
+                else rng.standard_normal(C).astype(np.float32))
+
+    rows.append(r(nan))
+    rows.append(r(-inf))
+    x = r(nan); x[C * 2 // 3] = -inf; rows.append(x)
+    x = r(-inf); x[::5] = nan; x[C - 2:] = inf; rows.append(x)
+    x = -np.abs(r()) - 1; x[C // 2] = -0.0; x[C // 3] = 0.0; rows.append(x)
+    x = r(); x[5 % C] = nan; rows.append(x)
+    x = r(); x[[C // 7, C // 2, C - 1]] = 9.0; rows.append(x)
+    x = r(); x[0] = 9.0; rows.append(x)
+    x = r(); x[C - 1] = 9.0; rows.append(x)
+    x = r(); x[min(3, C - 1)] = 9.0; x[C - 1] = 9.0; rows.append(x)
+    for _ in range(8):
+        rows.append(rng.integers(-2, 3, C).astype(np.float32))
+    vals = np.stack(rows)
+    full = np.concatenate([vals, rng.standard_normal((len(rows), pad)).astype(np.float32)], axis=1)
+    logits = torch.from_numpy(full).to(torch.bfloat16)   # all values exact in bf16
+    cu = wl.cu_seqlens([len(rows)])
+    _check(logits, cu, cuda_device, n_classes=C)

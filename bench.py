@@ -448,7 +448,47 @@ def run_nle(args, rank, world, local):
         del logits, flush
         torch.cuda.empty_cache()
 
+    # ---- full bidirectional attention over whole utterances (the encoder
+    # without blocks; the editor's attention) on the long-clip workload:
+    # 16 utterances of 1950-4700 frames, 16 heads x 64
+    va = None
+    if not args.no_varlen:
+        xv = wl.block_inputs(3, seed=wl.default_seed(3) + rank)
+        qv, kv, vv = (xv[n].to(dev) for n in ("q", "k", "v"))
+        cuv = torch.from_numpy(xv["cu"]).to(dev)
+        outv = torch.empty_like(qv)
+
+        def va_step():
+            nle.nle_varlen_attn_fwd(qv, kv, vv, outv, cuv, stream=sp)
+
+        for _ in range(3):
+            va_step()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        kv_reps = 20
+        a0.record(stream)
+        for _ in range(kv_reps):
+            va_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        va_ms = a0.elapsed_time(a1) / kv_reps
+        lens_v = [int(t) for t in xv["lengths"]]
+        hv_ = int(xv["heads"])
+        va_flops = 4 * D * hv_ * sum(t * t for t in lens_v)
+        va_bytes = 8 * D * hv_ * sum(lens_v)
+        va = {"workload": "long clips: 16 utterances of 1950-4700 frames (39-94 s at 50 Hz), 16 heads x 64, "
+                          "full attention inside each utterance",
+              "frames": int(sum(lens_v)), "ms": va_ms, "tflops": va_flops / (va_ms * 1e-3) / 1e12,
+              "algorithmic_flops": va_flops, "algorithmic_bytes": va_bytes,
+              "l2": "inputs ~0.32 GB > 126 MB L2; not flushed", "kernels": 1}
+        del qv, kv, vv, outv
+
     hbm_peak, tf_peak, tf_sust, peak_src = measured_peaks()
+    if va is not None:
+        va["pct_of_dense_bf16_peak"] = 100.0 * va["tflops"] / tf_peak
+        va["roofline"] = {"bound": "tensor", "achieved": va["tflops"], "peak": tf_peak, "unit": "TFLOP/s",
+                          "frac": va["tflops"] / tf_peak,
+                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json bf16_tflops)"}
     for extra in (pool, ctc):
         if extra is not None:
             extra["pct_of_hbm_peak"] = 100.0 * extra["gbs"] / hbm_peak
@@ -475,6 +515,7 @@ def run_nle(args, rank, world, local):
         "clocks": clocks.summary(),
         "e2e": {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ke},
+        "varlen_attn": va,
         "posterior_pool": pool,
         "ctc_decode": ctc,
         "gpu_launches": 2 * K * world,   # block + window kernel per step, all ranks
@@ -495,6 +536,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-ctc", action="store_true",
                     help="skip the pooling and CTC decoding measurements")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the full-utterance attention measurement")
     ap.add_argument("--ctc-utts", type=int, default=0,
                     help="pool and decode only the first N utterances (0: the whole batch)")
     args = ap.parse_args()

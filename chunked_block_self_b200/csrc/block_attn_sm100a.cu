@@ -51,6 +51,7 @@
 #include <cmath>
 
 #include "nle.h"
+#include "attn_softmax.cuh"
 #include "nle_device.cuh"
 #include "nle_host.h"
 
@@ -128,129 +129,6 @@ struct Params {
     unsigned long long wait_ns;
     int flags;
 };
-
-// Softmax of one TMEM lane quarter of a tile (32 rows, one per lane).
-//
-// In the log2 domain (x = s * scale * log2e) every p of a row is
-// exp2(x - m) for one shift m per row; softmax does not depend on m, which
-// only has to keep p in range.  m starts as the max of the row's first 16
-// keys, so the row's largest p is usually a small power above 1 (and exactly
-// 1 for a one-key block).  While p is formed, the largest exponent x - m of
-// the segment is tracked next to the exp; if any lane sees one above kYMax
-// (or a NaN), the warp takes the rare path: m moves up by a whole number k so
-// that the segment's max maps to 0, the segment is recomputed from the
-// registers that still hold it, and the P already written are rescaled by
-// 2^-k, an exact power of two.
-//
-// S is read from TMEM in register segments of SEG columns (a multiple of
-// 16, so each segment's P covers whole PV K-steps); each segment's exps are
-// one straight-line block.  P (bf16 pairs) is written back over S's first
-// columns.
-constexpr float kYMax = 32.f;
-
-template <int W, int N>
-__device__ __forceinline__ void seg_issue(uint32_t taddr, uint32_t (&s)[N])
-{
-    static_assert(W <= N && W % 16 == 0, "segment width");
-#pragma unroll
-    for (int c = 0; c + 32 <= W; c += 32)
-        tmem_ld32_nowait(taddr + c, &s[c]);
-    if constexpr (W % 32 == 16)
-        tmem_ld16_nowait(taddr + W - 16, &s[W - 16]);
-}
-
-template <int W, int N>
-__device__ __forceinline__ void seg_fence(uint32_t (&s)[N])
-{
-#pragma unroll
-    for (int i = 0; i < W; ++i)
-        reg_fence(s[i]);
-}
-
-template <int W>
-__device__ __forceinline__ void seg_store(uint32_t taddr, const uint32_t (&pk)[W / 2])
-{
-#pragma unroll
-    for (int c = 0; c + 32 <= W / 2; c += 32)
-        tmem_st32(taddr + c, &pk[c]);
-    if constexpr ((W / 2) % 32 >= 16)
-        tmem_st16p(taddr + (W / 2) / 32 * 32, &pk[(W / 2) / 32 * 32]);
-    if constexpr ((W / 2) % 16 == 8)
-        tmem_st8p(taddr + W / 2 - 8, &pk[W / 2 - 8]);
-}
-
-// Keys >= L (by index) -> -inf, branch-free (selects); only called for the
-// segment that holds L.
-template <int W, int N>
-__device__ __forceinline__ void seg_mask(uint32_t (&s)[N], int c0, int L)
-{
-#pragma unroll
-    for (int i = 0; i < W; ++i)
-        s[i] = c0 + i < L ? s[i] : __float_as_uint(-INFINITY);
-}
-
-// Exact max of the first W values (rare path and the initial shift).
-template <int W, int N>
-__device__ __forceinline__ float seg_max(const uint32_t (&s)[N])
-{
-    float mx[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-        mx[e] = fmaxf(__uint_as_float(s[e]), __uint_as_float(s[8 + e]));
-#pragma unroll
-    for (int i = 16; i + 16 <= W; i += 16)
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            mx[e] = fmax3(mx[e], __uint_as_float(s[i + e]), __uint_as_float(s[i + 8 + e]));
-    return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-}
-
-// p = exp2(s * sl2 - m) for the W keys (masked keys hold -inf -> 0), packed
-// to bf16 pairs; returns the segment sum, and the largest exponent in ymax.
-// Straight-line code: one basic block per segment keeps the exps of the
-// whole segment in flight.
-template <int W, int N>
-__device__ __forceinline__ float seg_exp(const uint32_t (&s)[N], uint32_t (&pk)[W / 2], float sl2, float m,
-                                         float &ymax)
-{
-    float ls[4] = {0.f, 0.f, 0.f, 0.f};
-    float ym[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-    for (int j = 0; j < W / 2; ++j) {
-        const float ya = fmaf(__uint_as_float(s[2 * j]), sl2, -m);
-        const float yb = fmaf(__uint_as_float(s[2 * j + 1]), sl2, -m);
-        ym[j & 3] = fmax3(ym[j & 3], ya, yb);
-        const float a = ex2_approx(ya);
-        const float b = ex2_approx(yb);
-        ls[j & 3] += a + b;
-        pk[j] = pack_bf16x2(a, b);
-    }
-    ymax = fmaxf(fmaxf(ym[0], ym[1]), fmaxf(ym[2], ym[3]));
-    return (ls[0] + ls[1]) + (ls[2] + ls[3]);
-}
-
-// Multiply the bf16 P already in TMEM columns [0, ncols) by f, a power of
-// two <= 1 (exact up to underflow); lanes with f = 1 rewrite P unchanged.
-// Rare path; must be entered by the whole warp.
-__device__ __forceinline__ void rescale_p(uint32_t tS, int ncols, float f)
-{
-    tmem_wait_st();
-    for (int c = 0; c < ncols; c += 8) {
-        uint32_t r[8];
-        tmem_ld8_nowait(tS + c, r);
-        tmem_wait_ld();
-        uint32_t o[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            reg_fence(r[i]);
-            const float a = __uint_as_float(r[i] << 16) * f;
-            const float b = __uint_as_float(r[i] & 0xffff0000u) * f;
-            o[i] = pack_bf16x2(a, b);
-        }
-        tmem_st8p(tS + c, o);
-        tmem_wait_st();
-    }
-}
 
 // Rare path of one segment (whole warp): S of the segment is still intact
 // in TMEM (its P has not been stored yet), so it is streamed again in

@@ -12,10 +12,9 @@
 // by its sum: no underflow when the blank dominates by far.
 //
 // One kernel, HBM-bound (reads each frame's hidden row and logits once,
-// writes each pooled row once).  A CTA takes whole windows: its warps reduce
-// the window's frames' logits (a warp per frame), then every thread forms
-// 8 output elements (one 16-byte chunk of the hidden dimension) from the
-// window's frames.
+// writes each pooled row once).  A warp takes whole windows: it reduces each
+// frame's logits to the frame's log weight, then every lane forms 8 output
+// elements (16-byte chunks of the hidden dimension) at a time.
 #include <climits>
 
 #include "nle.h"
@@ -64,89 +63,261 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
-// log(1 - p_blank) of one frame, on every lane of the warp (-inf: weight 0)
-__device__ __forceinline__ float frame_log_weight(const __nv_bfloat16 *__restrict__ z, int C, int lane)
+__device__ __forceinline__ void chunk_vals(const uint4 &q, float (&v)[8])
+{
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        v[2 * e] = __uint_as_float(w[e] << 16);
+        v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+    }
+}
+
+// log(1 - p_blank) of one frame, on every lane of the warp (-inf: weight 0).
+// With m the frame's largest logit, both sums are taken about m with one
+// exp per logit: log w = log sum_{c>=1} e^{z_c - m} - log sum_c e^{z_c - m}.
+// When the non-blank maximum mnb lies more than 60 below m (a blank that
+// dominates by far), the non-blank sum is taken again about mnb so that it
+// cannot underflow.  vec: rows 16-byte aligned and C a multiple of 8 (the
+// logits are read as 16-byte chunks of 8 classes).
+__device__ __forceinline__ float frame_log_weight(const __nv_bfloat16 *__restrict__ z, int C, bool vec, int lane)
 {
     float m = -INFINITY, mnb = -INFINITY;
-    for (int c = lane; c < C; c += 32) {
-        const float v = __bfloat162float(z[c]);
-        m = fmaxf(m, v);
-        if (c > 0)
-            mnb = fmaxf(mnb, v);
-    }
-    m = warp_max(m);
-    mnb = warp_max(mnb);
-    if (mnb == -INFINITY)
-        return -INFINITY;   // no non-blank class has any probability
-    // m >= mnb > -inf: both sums are >= 1 (their maximum term is 1)
     float s = 0.f, snb = 0.f;
-    for (int c = lane; c < C; c += 32) {
-        const float v = __bfloat162float(z[c]);
-        s += exp2f((v - m) * kLog2e);
-        if (c > 0)
-            snb += exp2f((v - mnb) * kLog2e);
+    if (vec && C <= 256) {
+        // at most one chunk per lane: the values stay in registers
+        float v[8];
+        const bool has = 8 * lane < C;
+        if (has) {
+            chunk_vals(__ldcs(reinterpret_cast<const uint4 *>(z) + lane), v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                m = fmaxf(m, v[e]);
+                if (lane > 0 || e > 0)
+                    mnb = fmaxf(mnb, v[e]);
+            }
+        }
+        m = warp_max(m);
+        mnb = warp_max(mnb);
+        if (mnb == -INFINITY)
+            return -INFINITY;   // no non-blank class has any probability
+        if (has) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float x = exp2f((v[e] - m) * kLog2e);
+                s += x;
+                if (lane > 0 || e > 0)
+                    snb += x;
+            }
+        }
+        if (mnb - m < -60.f) {
+            snb = 0.f;
+            if (has)
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (lane > 0 || e > 0)
+                        snb += exp2f((v[e] - mnb) * kLog2e);
+        }
+    } else if (vec) {
+        const uint4 *zc = reinterpret_cast<const uint4 *>(z);
+        for (int k = lane; 8 * k < C; k += 32) {
+            float v[8];
+            chunk_vals(zc[k], v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                m = fmaxf(m, v[e]);
+                if (k > 0 || e > 0)
+                    mnb = fmaxf(mnb, v[e]);
+            }
+        }
+        m = warp_max(m);
+        mnb = warp_max(mnb);
+        if (mnb == -INFINITY)
+            return -INFINITY;
+        const bool far = mnb - m < -60.f;   // warp-uniform
+        const float mr = far ? mnb : m;      // shift of the non-blank sum
+        for (int k = lane; 8 * k < C; k += 32) {
+            float v[8];
+            chunk_vals(zc[k], v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float x = exp2f((v[e] - m) * kLog2e);
+                s += x;
+                if (k > 0 || e > 0)
+                    snb += far ? exp2f((v[e] - mr) * kLog2e) : x;
+            }
+        }
+    } else {
+        for (int c = lane; c < C; c += 32) {
+            const float v = __bfloat162float(z[c]);
+            m = fmaxf(m, v);
+            if (c > 0)
+                mnb = fmaxf(mnb, v);
+        }
+        m = warp_max(m);
+        mnb = warp_max(mnb);
+        if (mnb == -INFINITY)
+            return -INFINITY;
+        const bool far = mnb - m < -60.f;
+        const float mr = far ? mnb : m;
+        for (int c = lane; c < C; c += 32) {
+            const float v = __bfloat162float(z[c]);
+            const float x = exp2f((v - m) * kLog2e);
+            s += x;
+            if (c > 0)
+                snb += far ? exp2f((v - mr) * kLog2e) : x;
+        }
     }
     s = warp_sum(s);
     snb = warp_sum(snb);
-    return (mnb - m) + (logf(snb) - logf(s));
+    // s >= 1 (its largest term is 1); snb > 0: mnb > -inf, and about mnb
+    // its largest term is 1
+    const float shift = mnb - m < -60.f ? mnb - m : 0.f;
+    return shift + (logf(snb) - logf(s));
 }
 
+// log(1 - p_blank) from one 16-byte logit chunk per lane already in
+// registers (rows 16-byte aligned, C a multiple of 8, C <= 256); the same
+// arithmetic as frame_log_weight's first branch.
+__device__ __forceinline__ float chunk_log_weight(const uint4 &q, int C, int lane)
+{
+    float v[8];
+    chunk_vals(q, v);
+    const bool has = 8 * lane < C;
+    float m = -INFINITY, mnb = -INFINITY;
+    if (has)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            m = fmaxf(m, v[e]);
+            if (lane > 0 || e > 0)
+                mnb = fmaxf(mnb, v[e]);
+        }
+    m = warp_max(m);
+    mnb = warp_max(mnb);
+    if (mnb == -INFINITY)
+        return -INFINITY;
+    const bool far = mnb - m < -60.f;
+    const float mr = far ? mnb : m;
+    float s = 0.f, snb = 0.f;
+    if (has)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float x = exp2f((v[e] - m) * kLog2e);
+            s += x;
+            if (lane > 0 || e > 0)
+                snb += far ? exp2f((v[e] - mr) * kLog2e) : x;
+        }
+    s = warp_sum(s);
+    snb = warp_sum(snb);
+    return (far ? mnb - m : 0.f) + (logf(snb) - logf(s));
+}
+
+constexpr int kPF = 2;   // frames of a window whose chunks are loaded up front
+constexpr int kCG = 4;   // hidden chunks per lane per group (128 chunks = 1024 columns)
+
+// One warp per window: the warp loads the first frames' hidden chunks and
+// logit chunks together, forms the weights, then pools.  No CTA-wide
+// barrier, so every warp keeps its own loads in flight.
 __global__ void __launch_bounds__(kPoolThreads) posterior_pool_kernel(PoolParams p)
 {
-    extern __shared__ float s_lw[];   // [P] log weights of the current window
+    extern __shared__ float s_lw_all[];   // [warps][P] log weights of each warp's window
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float *s_lw = s_lw_all + warp * p.P;
     const int n_chunks = p.dim >> 3;
+    const bool vec = (reinterpret_cast<uintptr_t>(p.logits) & 15) == 0 && (p.z_stride & 7) == 0 &&
+                     (p.n_classes & 7) == 0;
+    const bool zreg = vec && p.n_classes <= 256;
     PlanWalker w;
     w.init(p.cu, p.n_seq, p.total, p.P, lane);
-    for (long long g = blockIdx.x;; g += gridDim.x) {
+    const long long stride = (long long)gridDim.x * kPoolWarps;
+    for (long long g = (long long)blockIdx.x * kPoolWarps + warp;; g += stride) {
         int f0, L, seq;
         if (!w.find(g, lane, f0, L, seq))
             break;
         if (g >= p.n_rows) {
             // more windows than pooled rows: nothing past the buffer is written
-            if (tid == 0)
+            if (lane == 0)
                 report(p.status, NLE_ERR_INVALID_ARG);
             break;
         }
-        for (int t = warp; t < L; t += kPoolWarps) {
-            const float lw = frame_log_weight(p.logits + (long long)(f0 + t) * p.z_stride, p.n_classes, lane);
+        uint4 hv[kPF][kCG], zv[kPF];
+#pragma unroll
+        for (int t = 0; t < kPF; ++t) {
+            if (t < L) {
+                const __nv_bfloat16 *hrow = p.hidden + (long long)(f0 + t) * p.h_stride;
+#pragma unroll
+                for (int i = 0; i < kCG; ++i)
+                    if (lane + 32 * i < n_chunks)
+                        hv[t][i] = __ldcs(reinterpret_cast<const uint4 *>(hrow) + lane + 32 * i);
+                if (zreg && 8 * lane < p.n_classes)
+                    zv[t] = __ldcs(reinterpret_cast<const uint4 *>(p.logits + (long long)(f0 + t) * p.z_stride) +
+                                   lane);
+            }
+        }
+        float lw0 = -INFINITY;
+        for (int t = 0; t < L; ++t) {
+            float lw;
+            if (zreg && t < kPF)
+                lw = chunk_log_weight(t == 0 ? zv[0] : zv[kPF - 1], p.n_classes, lane);
+            else
+                lw = frame_log_weight(p.logits + (long long)(f0 + t) * p.z_stride, p.n_classes, vec, lane);
+            lw0 = fmaxf(lw0, lw);
             if (lane == 0) {
                 s_lw[t] = lw;
                 if (p.weights)
                     p.weights[f0 + t] = expf(lw);
             }
         }
-        __syncthreads();
-        float M = -INFINITY;
-        for (int t = 0; t < L; ++t)
-            M = fmaxf(M, s_lw[t]);
+        __syncwarp();
+        const float M = lw0;   // warp-uniform: every lane formed the same log weights
         __nv_bfloat16 *orow = p.pooled + g * (long long)p.dim;
-        for (int ch = tid; ch < n_chunks; ch += kPoolThreads) {
-            uint4 res = make_uint4(0u, 0u, 0u, 0u);
-            if (M != -INFINITY) {
-                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                float wsum = 0.f;
-                const __nv_bfloat16 *hrow = p.hidden + (long long)f0 * p.h_stride + 8 * ch;
-                for (int t = 0; t < L; ++t) {
-                    const float r = exp2f((s_lw[t] - M) * kLog2e);   // 0 for a weight of 0
-                    const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(hrow + (long long)t * p.h_stride));
-                    const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+        for (int cg = 0; 32 * kCG * cg < n_chunks; ++cg) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        acc[2 * e] = fmaf(r, __uint_as_float(wd[e] << 16), acc[2 * e]);
-                        acc[2 * e + 1] = fmaf(r, __uint_as_float(wd[e] & 0xffff0000u), acc[2 * e + 1]);
+            for (int i = 0; i < kCG; ++i) {
+                const int ch = 32 * kCG * cg + lane + 32 * i;
+                if (ch >= n_chunks)
+                    continue;
+                uint4 res = make_uint4(0u, 0u, 0u, 0u);
+                if (M != -INFINITY) {
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    float wsum = 0.f;
+#pragma unroll
+                    for (int t = 0; t < kPF; ++t) {
+                        if (t < L) {
+                            const float r = exp2f((s_lw[t] - M) * kLog2e);   // 0 for a weight of 0
+                            const uint4 q = cg == 0 ? hv[t][i]
+                                                    : __ldcs(reinterpret_cast<const uint4 *>(
+                                                                 p.hidden + (long long)(f0 + t) * p.h_stride) +
+                                                             ch);
+                            float v[8];
+                            chunk_vals(q, v);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                acc[e] = fmaf(r, v[e], acc[e]);
+                            wsum += r;
+                        }
                     }
-                    wsum += r;
+                    for (int t = kPF; t < L; ++t) {
+                        const float r = exp2f((s_lw[t] - M) * kLog2e);
+                        const uint4 q =
+                            __ldcs(reinterpret_cast<const uint4 *>(p.hidden + (long long)(f0 + t) * p.h_stride) + ch);
+                        float v[8];
+                        chunk_vals(q, v);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            acc[e] = fmaf(r, v[e], acc[e]);
+                        wsum += r;
+                    }
+                    const float inv = 1.f / wsum;   // wsum >= 1: the largest weight contributes 1
+                    res = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                                     pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
                 }
-                const float inv = 1.f / wsum;   // wsum >= 1: the largest weight contributes 1
-                res = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                                 pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+                *reinterpret_cast<uint4 *>(orow + 8 * ch) = res;
             }
-            *reinterpret_cast<uint4 *>(orow + 8 * ch) = res;
         }
-        __syncthreads();   // s_lw is rewritten by the next window
+        __syncwarp();   // s_lw is rewritten by the warp's next window
     }
-    if (w.bad && tid == 0)
+    if (w.bad && lane == 0)
         report(p.status, NLE_ERR_INVALID_ARG);
 }
 
@@ -191,8 +362,10 @@ extern "C" int nle_posterior_pool_fwd(const void *hidden, int64_t hidden_stride,
     p.pooled = static_cast<__nv_bfloat16 *>(pooled);
     p.weights = weights;
     p.status = dev_status;
-    const long long cap = (long long)di.sm_count * 16;
-    const int grid = (int)(n_pooled_rows < cap ? n_pooled_rows : cap);
-    posterior_pool_kernel<<<grid, kPoolThreads, sizeof(float) * pool_frames, static_cast<cudaStream_t>(stream)>>>(p);
+    // a warp per window; 4 CTAs of 128 threads fit an SM at 128 registers
+    const long long ctas = (n_pooled_rows + kPoolWarps - 1) / kPoolWarps, cap = (long long)di.sm_count * 4;
+    const int grid = (int)(ctas < cap ? ctas : cap);
+    posterior_pool_kernel<<<grid, kPoolThreads, sizeof(float) * kPoolWarps * pool_frames,
+                            static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
 }

@@ -57,6 +57,9 @@ _SIGS = {
     "nle_window_plan_host": ([_vp, _int, _int, _int, _vp, _vp, _vp, _vp, _vp, _int, ctypes.POINTER(_int)],
                              _int),
     "nle_shard_plan_host": ([_vp, _int, _int, _int, _vp], _int),
+    "nle_varlen_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _vp], _int),
+    "nle_varlen_attn_fwd_ex": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _f32, _i64, _vp, _int, _i64,
+                                _vp], _int),
     "nle_ctc_greedy_fwd": ([_vp, _i64, _int, _vp, _int, _i64, _vp, _vp, _vp, _vp], _int),
     "nle_posterior_pool_fwd": ([_vp, _i64, _int, _vp, _i64, _int, _vp, _int, _i64, _int, _i64, _vp, _vp, _vp,
                                 _vp], _int),
@@ -160,6 +163,47 @@ def block_attn(q, k, v, cu_seqlens, block_frames: int = 200, out=None, stream=No
     if out is None:
         out = torch.empty_like(q)
     nle_block_attn_fwd(q, k, v, out, cu_seqlens, block_frames=block_frames, stream=stream)
+    return out
+
+
+# ------------------------------------------------------------------ full-utterance attention
+def nle_varlen_attn_fwd(q, k, v, out, cu_seqlens, n_seq: int | None = None, total_frames: int | None = None,
+                        heads: int | None = None, d_head: int | None = None, stream=None) -> None:
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _dev_tensor(t, n, torch.bfloat16)
+    _dev_tensor(cu_seqlens, "cu_seqlens", torch.int32)
+    n_seq = cu_seqlens.numel() - 1 if n_seq is None else n_seq
+    total_frames = q.shape[0] if total_frames is None else total_frames
+    heads = q.shape[1] if heads is None else heads
+    d_head = q.shape[2] if d_head is None else d_head
+    _check(_lib.nle_varlen_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), n_seq,
+                                    total_frames, heads, d_head, _stream(stream)),
+           "nle_varlen_attn_fwd")
+
+
+def nle_varlen_attn_fwd_ex(q, k, v, out, cu_seqlens, n_seq: int | None = None, total_frames: int | None = None,
+                           heads: int | None = None, d_head: int = 64, softmax_scale: float = 0.0,
+                           row_stride_qkv: int = 0, dev_status=None, flags: int = 0, wait_limit_ns: int = 0,
+                           stream=None) -> None:
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _dev_tensor(t, n, torch.bfloat16)
+    _dev_tensor(cu_seqlens, "cu_seqlens", torch.int32)
+    if dev_status is not None:
+        _dev_tensor(dev_status, "dev_status", torch.int32)
+    n_seq = cu_seqlens.numel() - 1 if n_seq is None else n_seq
+    total_frames = out.shape[0] if total_frames is None else total_frames
+    heads = out.shape[1] if heads is None else heads
+    _check(_lib.nle_varlen_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), n_seq,
+                                       total_frames, heads, d_head, float(softmax_scale), row_stride_qkv,
+                                       _ptr(dev_status), flags, wait_limit_ns, _stream(stream)),
+           "nle_varlen_attn_fwd_ex")
+
+
+def varlen_attn(q, k, v, cu_seqlens, out=None, stream=None) -> torch.Tensor:
+    """O = full attention inside each packed utterance ([frames, heads, 64] bf16 CUDA)."""
+    if out is None:
+        out = torch.empty_like(q)
+    nle_varlen_attn_fwd(q, k, v, out, cu_seqlens, stream=stream)
     return out
 
 

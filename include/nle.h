@@ -148,6 +148,31 @@ int nle_window_xattn_fwd_ex(const void *q, const void *k, const void *v,
                             int64_t wait_limit_ns, void *stream);
 
 /* ---------------------------------------------------------------------
+ * Full bidirectional self-attention inside each packed utterance, any
+ * length (granite-speech-4.1-2b-nar model card, "Model Architecture" (3)
+ * Bidirectional LLM Editor: the LLM with its causal mask removed; "Usage /
+ * Installation": packed sequences, is_causal=False): for every utterance i
+ * and head h,  O = softmax(scale * Q K^T) V  over all T_i frames of the
+ * utterance -- block attention with one block per utterance.  Keys are
+ * walked in tiles of 128 with an online softmax (fp32, exact power-of-two
+ * rescaling), P rounded to bf16 before PV, O rounded to bf16.
+ *
+ * Arguments, layouts, ownership and errors as nle_block_attn_fwd, without
+ * block_frames (and no limit on T_i).  The _ex form adds softmax_scale
+ * (<= 0: 1/sqrt(d_head)), row_stride_qkv, dev_status, flags and the wait
+ * limit, as nle_block_attn_fwd_ex.
+ */
+int nle_varlen_attn_fwd(const void *q, const void *k, const void *v, void *out,
+                        const int32_t *cu_seqlens, int n_seq, int64_t total_frames,
+                        int heads, int d_head, void *stream);
+
+int nle_varlen_attn_fwd_ex(const void *q, const void *k, const void *v, void *out,
+                           const int32_t *cu_seqlens, int n_seq, int64_t total_frames,
+                           int heads, int d_head, float softmax_scale,
+                           int64_t row_stride_qkv, int32_t *dev_status, int flags,
+                           int64_t wait_limit_ns, void *stream);
+
+/* ---------------------------------------------------------------------
  * CTC greedy decoding of the encoder's CTC head (q4-RTN ONNX page,
  * "Inference note (NAR decode)"): the head emits n_classes per frame with
  * the blank at class 0, and a non-blank class c is token c - 1.  Per frame

@@ -7,42 +7,45 @@
 // the packed batch and every head,
 //     O = softmax(scale * Q K^T) V  over all T frames of the utterance.
 // The block kernel covers blocks of up to 256 frames in one key tile; here
-// the keys of an utterance are walked in tiles of 128 with an online
+// the keys of an utterance are walked in tiles of 64 with an online
 // softmax, so T is unbounded.
 //
-// Design (one persistent CTA per SM, 12 warps):
-//   warp 0      TMA producer.  Work item = (256 query rows of an utterance,
-//               head).  Per item it loads the item's Q (two 128-row boxes)
-//               into one of two Q stages, then every key tile of the
-//               utterance (K and V boxes of 128 rows) into a ring of KV
-//               stages, all 128-byte-swizzled (no multicast).
+// Design (one persistent CTA per SM, 20 warps):
+//   warp 0      TMA producer.  Work item = (512 query rows of an utterance,
+//               head).  Per item it loads the item's Q (one 128-row box
+//               per row tile that has rows) into one of two Q stages, then
+//               every key tile of the utterance (K and V boxes of 64 rows)
+//               into a ring of KV stages, all 128-byte-swizzled (no
+//               multicast).
 //   warp 1      owns TMEM (allocates and frees it).
 //   warp 2      V fix-up: waits for each KV stage to land and, for the
 //               utterance's last, partial key tile, zeroes V rows past the
 //               utterance up to the MMA's 16-row granule (their P is 0,
 //               but 0 * Inf would be NaN), then releases the stage to the
 //               chains.
-//   warps 4-7   chain 0: query rows 0..127 of the item, TMEM slot 0;
-//   warps 8-11  chain 1: rows 128..255, slot 1.  Both chains walk every
-//               key tile of the item, sharing the KV stages; their MMAs
-//               and softmaxes interleave (one's softmax runs while the
-//               tensor core works on the other's tile).  Per key tile j:
+//   warps 4-19  four chains of four warps; chain c takes query rows
+//               128c..128c+127 of the item in TMEM slot c.  All chains walk
+//               every key tile of the item, sharing the KV stages; their
+//               MMAs and softmaxes interleave, so the exp units always have
+//               rows to work on while other chains' MMAs run.  Per key
+//               tile j, the chain's first warp issues (one elected lane):
 //                 S = Q_c K_j^T  (tcgen05.mma kind::f16, M=128,
 //                                N=ceil16(valid keys), K=64 in 4 steps)
-//                 softmax: p = exp2(S*scale*log2e - m) with the row's
-//                   running shift m (set from the first 16 keys of the
-//                   first tile); keys past the utterance are 0 by index.
-//                   If an exponent would exceed 32, m moves up by a whole
-//                   k and the row's P, running sum and O are scaled by 2^-k
-//                   (exact).  P (bf16) is written over S.
+//               and, once its four warps have written P,
 //                 O += P V_j     (A = P from TMEM, B = V_j N-major, M=128,
-//                                N=64, K=ceil16(valid keys))
+//                                N=64, K=ceil16(valid keys)).
+//               softmax: p = exp2(S*scale*log2e - m) with the row's running
+//               shift m (set from the first 16 keys of the first tile) in
+//               32-column register segments; keys past the utterance are 0
+//               by index.  If an exponent would exceed 32, m moves up by a
+//               whole k and the row's P, running sum and O are scaled by
+//               2^-k (exact).  P (bf16) is written over S.
 //               After the last tile O is read, divided by the row sum,
 //               rounded to bf16 and stored with 16-byte stores, rows of the
-//               utterance only.  A chain with no rows in the item (an item
-//               of <= 128 rows) only releases the item's stages.
-// TMEM (512 columns): slot c at column 256*c holds S (128 columns; P over
-// its first 64) and O (64 columns at +128).
+//               utterance only.  A chain with no rows in the item only
+//               releases the item's stages.
+// TMEM (512 columns): slot c at column 128*c holds S (64 columns; P over
+// its first 32) and O (64 columns at +64).
 //
 // Every mbarrier wait is bounded; on expiry the CTA drains its copies and
 // MMAs in flight, frees TMEM and returns.
@@ -57,30 +60,33 @@ namespace {
 
 using namespace nle;
 
-constexpr int kThreads = 384;
-constexpr int kChain0 = 4;                          // first warp of chain 0
-constexpr int kTile = 128;                          // query rows per chain; keys per key tile
-constexpr int kPair = 2 * kTile;                    // query rows per item
-constexpr int kRowBytes = 128;                      // one frame of one head: 64 bf16
-constexpr uint32_t kTileBytes = kTile * kRowBytes;  // 16 KB
-constexpr uint32_t kQStageBytes = 2 * kTileBytes;
-constexpr uint32_t kKVStageBytes = 2 * kTileBytes;  // K, then V
-constexpr int kMaxKV = 8;
+constexpr int kChains = 4;                                  // softmax chains of 128 query rows
+constexpr int kChain0 = 4;                                  // first warp of chain 0
+constexpr int kThreads = 32 * (kChain0 + 4 * kChains);      // 640
+constexpr int kQRows = 128;                                 // query rows per chain (MMA M)
+constexpr int kItemRows = kChains * kQRows;                 // query rows per item
+constexpr int kKeys = 64;                                   // keys per KV tile (one S/PV round)
+constexpr int kRowBytes = 128;                              // one frame of one head: 64 bf16
+constexpr uint32_t kQTileBytes = kQRows * kRowBytes;        // 16 KB
+constexpr uint32_t kQStageBytes = kChains * kQTileBytes;    // 64 KB
+constexpr uint32_t kKVTileBytes = kKeys * kRowBytes;        // 8 KB
+constexpr uint32_t kKVStageBytes = 2 * kKVTileBytes;        // K, then V
+constexpr int kMaxKV = 12;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSlotCols = 256;
-constexpr uint32_t kOCol = 128;
-constexpr int kSeg = 64;                            // softmax register segment (2 per key tile)
+constexpr uint32_t kSlotCols = 128;                         // per chain: S (64 columns), then O
+constexpr uint32_t kOCol = 64;
+constexpr int kSeg = 32;                                    // softmax register segment (2 per key tile)
 
 struct Bars {
     uint64_t q_full[2];
-    uint64_t q_empty[2];         // 2 arrivals: each chain's last S MMA of the item
+    uint64_t q_empty[2];         // kChains arrivals: each chain's last S MMA of the item
     uint64_t kv_full[kMaxKV];
     uint64_t kv_ready[kMaxKV];   // the fix-up warp has checked the stage
-    uint64_t kv_empty[kMaxKV];   // 2 arrivals: each chain's PV MMA of the tile
-    uint64_t s_full[2];
-    uint64_t wg_p[2];            // 4 arrivals: P of the tile written
-    uint64_t o_done[2];          // the chain's latest PV MMA has completed
-    uint64_t mma_done[2];
+    uint64_t kv_empty[kMaxKV];   // kChains arrivals: each chain's PV MMA of the tile
+    uint64_t s_full[kChains];
+    uint64_t wg_p[kChains];      // 4 arrivals: P of the tile written
+    uint64_t o_done[kChains];    // the chain's latest PV MMA has completed
+    uint64_t mma_done[kChains];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -102,7 +108,7 @@ struct Params {
 };
 
 // The CTA's items in order: item i = blockIdx.x + n * gridDim.x = u * H + h,
-// u = the 256-row query unit of the batch.  Every role walks the same
+// u = the 512-row query unit of the batch.  Every role walks the same
 // sequence.
 struct ItemWalk {
     PlanWalker w;
@@ -110,7 +116,7 @@ struct ItemWalk {
 
     __device__ __forceinline__ void init(const Params &p, int lane)
     {
-        w.init(p.cu, p.n_seq, p.total, kPair, lane);
+        w.init(p.cu, p.n_seq, p.total, kItemRows, lane);
         H = p.heads;
         b = (int)(blockIdx.x / H);
         h = (int)(blockIdx.x % H);
@@ -247,14 +253,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_u32(&bars->q_full[s]), 1);
-            mbar_init(smem_u32(&bars->q_empty[s]), 2);
+            mbar_init(smem_u32(&bars->q_empty[s]), kChains);
         }
         for (int s = 0; s < nkv; ++s) {
             mbar_init(smem_u32(&bars->kv_full[s]), 1);
             mbar_init(smem_u32(&bars->kv_ready[s]), 1);
-            mbar_init(smem_u32(&bars->kv_empty[s]), 2);
+            mbar_init(smem_u32(&bars->kv_empty[s]), kChains);
         }
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < kChains; ++c) {
             mbar_init(smem_u32(&bars->s_full[c]), 1);
             mbar_init(smem_u32(&bars->wg_p[c]), 4);
             mbar_init(smem_u32(&bars->o_done[c]), 1);
@@ -299,14 +305,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0 && !(skip0 && nq == 0)) {
                 const uint32_t bar = smem_u32(&bars->q_full[qs]);
                 const uint32_t dst = q_base + qs * kQStageBytes;
-                mbar_arrive_expect_tx(bar, (L > kTile ? 2u : 1u) * kTileBytes);
-                tma_load_2d(dst, &tm_q, h * 64, f0, bar, pol_q);
-                if (L > kTile)
-                    tma_load_2d(dst + kTileBytes, &tm_q, h * 64, f0 + kTile, bar, pol_q);
+                const int boxes = (L + kQRows - 1) / kQRows;   // row tiles with query rows
+                mbar_arrive_expect_tx(bar, (uint32_t)boxes * kQTileBytes);
+                for (int c = 0; c < boxes; ++c)
+                    tma_load_2d(dst + c * kQTileBytes, &tm_q, h * 64, f0 + c * kQRows, bar, pol_q);
             }
             __syncwarp();
             ++nq;
-            for (int j = 0; j * kTile < T; ++j) {
+            for (int j = 0; j * kKeys < T; ++j) {
                 const int s = nkt % nkv;
                 const uint32_t u = (uint32_t)(nkt / nkv);
                 if (u > 0 &&
@@ -317,9 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
                     const uint32_t bar = smem_u32(&bars->kv_full[s]);
                     const uint32_t dst = kv_base + s * kKVStageBytes;
-                    mbar_arrive_expect_tx(bar, 2u * kTileBytes);
-                    tma_load_2d_nohint(dst, &tm_k, h * 64, us + j * kTile, bar);
-                    tma_load_2d_nohint(dst + kTileBytes, &tm_v, h * 64, us + j * kTile, bar);
+                    mbar_arrive_expect_tx(bar, kKVStageBytes);
+                    tma_load_2d_nohint(dst, &tm_k, h * 64, us + j * kKeys, bar);
+                    tma_load_2d_nohint(dst + kKVTileBytes, &tm_v, h * 64, us + j * kKeys, bar);
                 }
                 __syncwarp();
                 ++nkt;
@@ -349,17 +355,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             int f0, L, us, T, h;
             if (!it.next(p, lane, f0, L, us, T, h))
                 break;
-            for (int j = 0; j * kTile < T; ++j, ++nkt) {
+            for (int j = 0; j * kKeys < T; ++j, ++nkt) {
                 const int s = nkt % nkv;
                 if (!wait_bar(smem_u32(&bars->kv_full[s]), (uint32_t)(nkt / nkv) & 1, abort_flag, wait_ns,
                               p.status)) {
                     stop = true;
                     break;
                 }
-                const int nv = T - j * kTile < kTile ? T - j * kTile : kTile;
+                const int nv = T - j * kKeys < kKeys ? T - j * kKeys : kKeys;
                 const int nk = (nv + 15) & ~15;
                 if (nv < nk) {
-                    uint4 *vz = reinterpret_cast<uint4 *>(smem + p.kv_off + s * kKVStageBytes + kTileBytes +
+                    uint4 *vz = reinterpret_cast<uint4 *>(smem + p.kv_off + s * kKVStageBytes + kKVTileBytes +
                                                           nv * kRowBytes);
                     for (int i = lane; i < (nk - nv) * (kRowBytes / 16); i += 32)
                         vz[i] = make_uint4(0, 0, 0, 0);
@@ -392,9 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!it.next(p, lane, f0, L, us, T, h))
                 break;
             const int qs = n & 1;
-            const int tiles = (T + kTile - 1) / kTile;
-            const bool chain_rows = L > c * kTile;
-            const int row0 = c * kTile + qq * 32;   // first item row of this warp
+            const int tiles = (T + kKeys - 1) / kKeys;
+            const bool chain_rows = L > c * kQRows;
+            const int row0 = c * kQRows + qq * 32;   // first item row of this warp
             const bool active = row0 < L;
             if (leader &&
                 !wait_bar(smem_u32(&bars->q_full[qs]), (uint32_t)(n >> 1) & 1, abort_flag, wait_ns, p.status)) {
@@ -425,10 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 continue;
             }
             float m = 0.f, l = 0.f;
-            const uint32_t qaddr = q_base + qs * kQStageBytes + c * kTileBytes;
+            const uint32_t qaddr = q_base + qs * kQStageBytes + c * kQTileBytes;
             for (int j = 0; j < tiles; ++j, ++nkt) {
                 const int s = nkt % nkv;
-                const int nv = T - j * kTile < kTile ? T - j * kTile : kTile;
+                const int nv = T - j * kKeys < kKeys ? T - j * kKeys : kKeys;
                 const int nk = (nv + 15) & ~15;
                 const uint32_t kaddr = kv_base + s * kKVStageBytes;
                 // ---------------------------------------------- S = Q K^T
@@ -483,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                         // N = 64 is one 128-byte swizzle atom along N; K
                         // steps of 16 rows advance the start by 2048 bytes
-                        const uint64_t dv = smem_desc_sw128(kaddr + kTileBytes, 0, 1024);
+                        const uint64_t dv = smem_desc_sw128(kaddr + kKVTileBytes, 0, 1024);
                         if (elect_one()) {
                             for (int kk = 0; kk < nk / 16; ++kk)
                                 mma_ts(slot + kOCol, slot + kk * 8, dv + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
@@ -507,27 +513,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             if (active) {
-                uint32_t o[64];
-#pragma unroll
-                for (int cc = 0; cc < 64; cc += 16)
-                    tmem_ld16_nowait(tS + kOCol + cc, &o[cc]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    reg_fence(o[i]);
+                // O in two halves of 32 columns (registers are scarce at 20 warps)
                 const float inv = 1.f / l;
-                if (row0 + lane < L) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (size_t)(f0 + row0 + lane) * p.out_stride + h * 64);
+                const bool row_ok = row0 + lane < L;
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (size_t)(f0 + row0 + lane) * p.out_stride + h * 64);
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc)
-                        dst[cc] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * cc]) * inv,
-                                                         __uint_as_float(o[8 * cc + 1]) * inv),
-                                             pack_bf16x2(__uint_as_float(o[8 * cc + 2]) * inv,
-                                                         __uint_as_float(o[8 * cc + 3]) * inv),
-                                             pack_bf16x2(__uint_as_float(o[8 * cc + 4]) * inv,
-                                                         __uint_as_float(o[8 * cc + 5]) * inv),
-                                             pack_bf16x2(__uint_as_float(o[8 * cc + 6]) * inv,
-                                                         __uint_as_float(o[8 * cc + 7]) * inv));
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t o[32];
+                    tmem_ld32_nowait(tS + kOCol + 32 * half, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        reg_fence(o[i]);
+                    if (row_ok) {
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc)
+                            dst[4 * half + cc] = make_uint4(
+                                pack_bf16x2(__uint_as_float(o[8 * cc]) * inv, __uint_as_float(o[8 * cc + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * cc + 2]) * inv, __uint_as_float(o[8 * cc + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * cc + 4]) * inv, __uint_as_float(o[8 * cc + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * cc + 6]) * inv, __uint_as_float(o[8 * cc + 7]) * inv));
+                    }
                 }
             }
             tc_fence_before();
@@ -566,8 +572,8 @@ extern "C" int nle_varlen_attn_fwd_ex(const void *q, const void *k, const void *
         return NLE_ERR_INVALID_ARG;
     if (d_head != 64 || total_frames > 0x7fffffffLL)
         return NLE_ERR_UNSUPPORTED;
-    // upper bound on work items: each utterance has at most T/256 + 1 query units
-    const long long max_items = ((long long)n_seq + total_frames / kPair) * heads;
+    // upper bound on work items: each utterance has at most T/512 + 1 query units
+    const long long max_items = ((long long)n_seq + total_frames / kItemRows) * heads;
     if (max_items > 0x7fffffffLL)
         return NLE_ERR_UNSUPPORTED;
     if (n_seq == 0 || total_frames == 0)
@@ -590,7 +596,7 @@ extern "C" int nle_varlen_attn_fwd_ex(const void *q, const void *k, const void *
         return NLE_ERR_UNSUPPORTED;
     // the kernel counts the key tiles a CTA walks in 32 bits
     const long long grid_ll = max_items < di.sm_count ? max_items : di.sm_count;
-    if ((max_items / grid_ll + 1) * (total_frames / kTile + 1) > 0x7fffffffLL)
+    if ((max_items / grid_ll + 1) * (total_frames / kKeys + 1) > 0x7fffffffLL)
         return NLE_ERR_UNSUPPORTED;
 
     Params p{};
@@ -624,9 +630,9 @@ extern "C" int nle_varlen_attn_fwd_ex(const void *q, const void *k, const void *
 
     CUtensorMap tq, tk, tv;
     const uint64_t cols = (uint64_t)dense, rows = (uint64_t)total_frames;
-    if (!nle::encode_tmap_bf16_2d(&tq, q, cols, rows, stride, 64, kTile) ||
-        !nle::encode_tmap_bf16_2d(&tk, k, cols, rows, stride, 64, kTile) ||
-        !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, stride, 64, kTile))
+    if (!nle::encode_tmap_bf16_2d(&tq, q, cols, rows, stride, 64, kQRows) ||
+        !nle::encode_tmap_bf16_2d(&tk, k, cols, rows, stride, 64, kKeys) ||
+        !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, stride, 64, kKeys))
         return NLE_ERR_CUDA;
 
     const int slot = dev < 64 ? dev : 0;

@@ -48,12 +48,21 @@ B, W, QW, D = 200, 15, 3, 64
 # (reported as null once the source changes).  Read below 1.0: part of the
 # output is still dirty in the 126 MB L2 when the launch ends.
 NCU_TRAFFIC = {
-    "block_attn": {"files": ("block_attn_sm100a.cu", "nle_device.cuh"),
-                   "source_sha256": "28408a1de518a6d1155e74dc3ef6b2177e97d019409ea5f35d620b980ff6fa4a",
-                   "traffic_over_algorithmic": (376876032 + 67080960) / 482533376},
+    "block_attn": {"files": ("block_attn_sm100a.cu", "attn_softmax.cuh", "nle_device.cuh"),
+                   "source_sha256": "08a3ba5e183344821f7885269daca4c1af162b4915e67500ba2647da98e9f57f",
+                   "traffic_over_algorithmic": (378200320 + 67069440) / 482533376},
     "window_xattn": {"files": ("window_xattn_sm100a.cu", "nle_device.cuh"),
                      "source_sha256": "33de401559e416ea91ea8b491baed1a3b0d3db061b0ad53ff9b193776c55bc03",
                      "traffic_over_algorithmic": (265945600 + 7834112) / 290320384},
+    # full-utterance attention: the long-clip workload, the same launch as the bench's
+    "varlen_attn": {"files": ("varlen_attn_sm100a.cu", "attn_softmax.cuh", "nle_device.cuh"),
+                    "source_sha256": "c23de0a8c69781ae4e1d73eb1a3fce330b1fd2a31b11bd97d4cbab9eb381330d",
+                    "traffic_over_algorithmic": (342620416 + 90884608) / 439304192},
+    # CTC argmax: captured on 16 utterances (3,300 rows, 662.4 MB); traffic grows
+    # with rows, so the ratio is applied to the full batch
+    "ctc_argmax": {"files": ("ctc_sm100a.cu", "nle_device.cuh"),
+                   "source_sha256": "e535a0a83de57f00c0ae4d914ea66fc8ca060f95811011549aae132f9a3f833e",
+                   "traffic_over_algorithmic": (739151872 + 6230272) / 662369464},
 }
 
 
@@ -444,7 +453,9 @@ def run_nle(args, rank, world, local):
         ctc_bytes = logits.numel() * 2 + n_rows * 12 + len(clen) * 4
         ctc = {"rows": n_rows, "utterances": len(clen), "classes": int(logits.shape[1]), "ms": ctc_ms,
                "rows_per_s": n_rows / (ctc_ms * 1e-3), "gbs": ctc_bytes / (ctc_ms * 1e-3) / 1e9,
-               "algorithmic_bytes": ctc_bytes, "l2": "flushed (256 MB write) before each launch", "kernels": 2}
+               "algorithmic_bytes": ctc_bytes, "l2": "flushed (256 MB write) before each launch", "kernels": 2,
+               # the argmax kernel's DRAM bytes (logits once, classes written)
+               "traffic_argmax": ncu_traffic("ctc_argmax", logits.numel() * 2 + n_rows * 4)}
         del logits, flush
         torch.cuda.empty_cache()
 
@@ -480,7 +491,8 @@ def run_nle(args, rank, world, local):
                           "full attention inside each utterance",
               "frames": int(sum(lens_v)), "ms": va_ms, "tflops": va_flops / (va_ms * 1e-3) / 1e12,
               "algorithmic_flops": va_flops, "algorithmic_bytes": va_bytes,
-              "l2": "inputs ~0.32 GB > 126 MB L2; not flushed", "kernels": 1}
+              "l2": "inputs ~0.32 GB > 126 MB L2; not flushed", "kernels": 1,
+              "traffic": ncu_traffic("varlen_attn", va_bytes)}
         del qv, kv, vv, outv
 
     hbm_peak, tf_peak, tf_sust, peak_src = measured_peaks()

@@ -49,20 +49,20 @@ B, W, QW, D = 200, 15, 3, 64
 # output is still dirty in the 126 MB L2 when the launch ends.
 NCU_TRAFFIC = {
     "block_attn": {"files": ("block_attn_sm100a.cu", "attn_softmax.cuh", "nle_device.cuh"),
-                   "source_sha256": "08a3ba5e183344821f7885269daca4c1af162b4915e67500ba2647da98e9f57f",
-                   "traffic_over_algorithmic": (378200320 + 67069440) / 482533376},
+                   "source_sha256": "2e6ebd9f63407760f95d35cad80618ba9226f66a254b7f3478e5c0a62b707595",
+                   "traffic_over_algorithmic": (377232640 + 66526720) / 482533376},
     "window_xattn": {"files": ("window_xattn_sm100a.cu", "nle_device.cuh"),
-                     "source_sha256": "33de401559e416ea91ea8b491baed1a3b0d3db061b0ad53ff9b193776c55bc03",
-                     "traffic_over_algorithmic": (265945600 + 7834112) / 290320384},
+                     "source_sha256": "43ecd044325aac9d122bc38ba666274726781c3720caf2f2a5fcb5b34fb21737",
+                     "traffic_over_algorithmic": (265946112 + 7618304) / 290320384},
     # full-utterance attention: the long-clip workload, the same launch as the bench's
     "varlen_attn": {"files": ("varlen_attn_sm100a.cu", "attn_softmax.cuh", "nle_device.cuh"),
-                    "source_sha256": "c23de0a8c69781ae4e1d73eb1a3fce330b1fd2a31b11bd97d4cbab9eb381330d",
-                    "traffic_over_algorithmic": (342620416 + 90884608) / 439304192},
+                    "source_sha256": "f97abe68c26d62ac374fa754a2f1b1536b5e4cc4598e43d5712680b93a44f41f",
+                    "traffic_over_algorithmic": (343228160 + 91153152) / 439304192},
     # CTC argmax: captured on 16 utterances (3,300 rows, 662.4 MB); traffic grows
     # with rows, so the ratio is applied to the full batch
     "ctc_argmax": {"files": ("ctc_sm100a.cu", "nle_device.cuh"),
-                   "source_sha256": "e535a0a83de57f00c0ae4d914ea66fc8ca060f95811011549aae132f9a3f833e",
-                   "traffic_over_algorithmic": (739151872 + 6230272) / 662369464},
+                   "source_sha256": "dc0ebd4500f03c2450606136a33502b06bc01edfa47d3ad49651a89a64928637",
+                   "traffic_over_algorithmic": (739271680 + 3598336) / 662369464},
 }
 
 

@@ -267,3 +267,4 @@ def threads_used(n_threads: int = 0) -> int:
 from .ctc import collapse as ctc_collapse, ctc_greedy, frame_classes as ctc_frame_classes  # noqa: E402,F401
 from .pool import (blank_weights, log_weights as pool_log_weights,  # noqa: E402,F401
                    pooled_rows, posterior_pool)
+from .qkv import block_attn_f64, block_attn_qkv, qkv_project  # noqa: E402,F401

@@ -8,12 +8,18 @@ library (for instance to draw inputs on a CPU-only host).
 """
 __all__ = ["nle", "workloads"]
 
+_SUBMODULES = ("nle", "workloads", "build", "dp")
+
 
 def __getattr__(name):
-    if name in ("nle", "workloads"):
-        import importlib
+    import importlib
+    # submodules first: `build` and `workloads` must import without the
+    # CUDA library (the build creates it)
+    if name in _SUBMODULES:
         return importlib.import_module(f"{__name__}.{name}")
-    from . import nle as _nle
+    if name.startswith("_"):
+        raise AttributeError(name)
+    _nle = importlib.import_module(f"{__name__}.nle")
     if hasattr(_nle, name):
         return getattr(_nle, name)
     raise AttributeError(name)

@@ -1,6 +1,8 @@
 /*
  * nle.h -- C ABI of libnle.so: varlen block self-attention and windowed
- * cross-attention on NVIDIA B200 (sm_100a).
+ * cross-attention on NVIDIA B200 (sm_100a), with full-utterance attention,
+ * the BPE head's posterior-weighted pooling and CTC greedy decoding (each
+ * documented at its entry point below).
  *
  * The operations (sources are the web pages this library follows):
  *
@@ -21,7 +23,8 @@
  *  queries_per_window*g ... +queries_per_window-1, each attending to the
  *  window's frames.
  *
- * Conventions for every entry point below:
+ * Conventions for every attention entry point below (the pooling and CTC
+ * entry points state their own layouts):
  *  - Tensor pointers (q, k, v, out, cu_seqlens, dev_status) are DEVICE
  *    pointers owned by the caller.  The library never allocates, frees or
  *    synchronises; every launch is asynchronous on `stream` (a cudaStream_t;

@@ -34,16 +34,28 @@ def _as_f64(logits) -> np.ndarray:
     return a.astype(np.float64)
 
 
-def frame_classes(logits) -> np.ndarray:
+def frame_classes(logits, rows_per_pass: int = 256) -> np.ndarray:
     """Class of the largest logit of each frame ([T, C] -> [T] int64): the
     first (lowest) class among equal maxima, NaN logits skipped, the blank
-    when a frame has no other candidate."""
-    x = _as_f64(logits)
-    out = np.zeros(x.shape[0], np.int64)
-    for t in range(x.shape[0]):
-        ok = np.nonzero(~np.isnan(x[t]))[0]   # the candidate classes, ascending
-        if ok.size:
-            out[t] = ok[np.argmax(x[t, ok])]   # first (lowest) of the maxima
+    when a frame has no other candidate.
+
+    Written with whole-array operations over ``rows_per_pass`` frames at a
+    time (the definition is per frame; passes only bound the memory)."""
+    try:
+        import torch
+        if isinstance(logits, torch.Tensor):
+            logits = logits.contiguous().view(torch.int16).numpy().view(np.uint16)
+    except ImportError:
+        pass
+    src = np.asarray(logits)
+    out = np.zeros(src.shape[0], np.int64)
+    for a in range(0, src.shape[0], rows_per_pass):
+        x = _as_f64(src[a:a + rows_per_pass])
+        cand = ~np.isnan(x)                                   # the candidate classes
+        best = np.where(cand, x, -np.inf).max(axis=1, initial=-np.inf)
+        hit = cand & (x == best[:, None])                     # candidates holding the maximum
+        any_hit = hit.any(axis=1)
+        out[a:a + x.shape[0]] = np.where(any_hit, hit.argmax(axis=1), 0)   # lowest such class
     return out
 
 

@@ -97,3 +97,29 @@ NONFINITE = [
 @pytest.mark.parametrize("row,cls", NONFINITE)
 def test_nonfinite_and_signed_zero(row, cls):
     assert oracle.ctc_frame_classes(_bf16_bits([row])).tolist() == [cls]
+
+
+def _brute_force_class(row):
+    """Per-frame class by a plain scan: the first non-NaN logit that no later
+    non-NaN logit exceeds (strictly), the blank when every logit is NaN."""
+    best, cls = None, 0
+    for c, z in enumerate(row):
+        if z != z:          # NaN: no candidate
+            continue
+        if best is None or z > best:
+            best, cls = z, c
+    return cls
+
+
+def test_frame_classes_match_a_plain_scan_on_small_rows():
+    """The array formulation against a pure-Python scan on tiny rows that mix
+    NaN, +-inf, -0/+0 and ties, over several pass sizes (including rows
+    split across passes)."""
+    rng = np.random.default_rng(17)
+    pool = np.array([np.nan, np.inf, -np.inf, -0.0, 0.0, 1.0, -1.0, 2.0], np.float32)
+    for n_cls in (1, 2, 3, 5, 9):
+        vals = rng.choice(pool, size=(64, n_cls))
+        want = [_brute_force_class(r.tolist()) for r in vals]
+        for per_pass in (1, 7, 256):
+            got = oracle.ctc_frame_classes(_bf16_bits(vals), rows_per_pass=per_pass)
+            assert got.tolist() == want

@@ -633,9 +633,6 @@ KernelInfo pick_kernel(int nb)
     }
 }
 
-// Per (NB/16, device): dynamic smem opted in so far.
-int g_smem_set[17][64] = {};
-
 } // namespace
 
 extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v, void *out,
@@ -731,14 +728,8 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
         return NLE_ERR_CUDA;
 
     const KernelInfo kern = pick_kernel(NB);
-    const int slot = dev < 64 ? dev : 0;
-    int &set = g_smem_set[NB / 16][slot];
-    if (dev >= 64 || set < (int)smem) {
-        if (cudaFuncSetAttribute(reinterpret_cast<const void *>(kern.fn),
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return NLE_ERR_CUDA;
-        set = (int)smem;
-    }
+    if (!nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(kern.fn), dev, di.smem_optin))
+        return NLE_ERR_CUDA;
     const int grid = (int)(max_items < di.sm_count ? max_items : di.sm_count);
     kern.fn<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tq0, tq1, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;

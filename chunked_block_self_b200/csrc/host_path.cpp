@@ -151,12 +151,13 @@ extern "C" int nle_path_fwd_host(const nle_path_buffers *b, int n_seq, int64_t t
         // the chunk's slice of cu keeps absolute frame offsets; the window
         // kernel numbers the chunk's windows from 0, so its query and output
         // pointers start at the chunk's first query row
-        rc = nle_block_attn_fwd(b->d_q, b->d_k, b->d_v, b->d_out, b->d_cu + i0, i1 - i0, total_frames, heads,
-                                d_head, block_frames, s);
+        rc = nle_block_attn_fwd_ex(b->d_q, b->d_k, b->d_v, b->d_out, b->d_cu + i0, i1 - i0, total_frames, heads,
+                                   d_head, block_frames, 0.f, 0, b->d_status, 0, 0, s);
         if (rc != NLE_OK)
             break;
-        rc = nle_window_xattn_fwd(at(b->d_qw, r0, row_bytes), b->d_kw, b->d_vw, at(b->d_out_w, r0, row_bytes),
-                                  b->d_cu + i0, i1 - i0, total_frames, nr, heads, d_head, window_frames, Qw, s);
+        rc = nle_window_xattn_fwd_ex(at(b->d_qw, r0, row_bytes), b->d_kw, b->d_vw, at(b->d_out_w, r0, row_bytes),
+                                     b->d_cu + i0, i1 - i0, total_frames, nr, heads, d_head, window_frames, Qw, 0.f,
+                                     b->d_status, 0, 0, s);
         if (rc != NLE_OK)
             break;
         if ((nf > 0 && cudaMemcpyAsync(at(b->out, f0, row_bytes), at(static_cast<const void *>(b->d_out), f0,

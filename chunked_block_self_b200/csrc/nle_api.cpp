@@ -2,6 +2,8 @@
 // tensor-map encoder (cuTensorMapEncodeTiled reached through the runtime's
 // driver entry point, so libnle.so does not link libcuda directly).
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "nle.h"
 #include "nle_host.h"
@@ -61,6 +63,19 @@ bool current_device_info(DeviceInfo *info, int *device)
     g_info[dev] = d;
     g_have[dev] = true;
     *info = d;
+    return true;
+}
+
+bool allow_max_dynamic_smem(const void *fn, int device, int smem_optin)
+{
+    static std::mutex mu;
+    static std::set<std::pair<const void *, int>> done;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({fn, device}))
+        return true;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin) != cudaSuccess)
+        return false;
+    done.insert({fn, device});
     return true;
 }
 

@@ -29,6 +29,13 @@ bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t cols, uint
 bool encode_tmap_bf16_heads(CUtensorMap *map, const void *base, uint64_t rows, uint64_t heads,
                             uint64_t row_stride_elems, uint32_t box_rows, uint32_t box_heads);
 
+// Lets `fn` launch with any dynamic shared memory size up to the device's
+// opt-in maximum (cudaFuncAttributeMaxDynamicSharedMemorySize set once per
+// kernel and device, under a lock; the attribute only ever grows, so
+// concurrent callers cannot undo each other).  Returns false if the CUDA
+// call fails.
+bool allow_max_dynamic_smem(const void *fn, int device, int smem_optin);
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 } // namespace nle

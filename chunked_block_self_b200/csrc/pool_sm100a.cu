@@ -365,7 +365,12 @@ extern "C" int nle_posterior_pool_fwd(const void *hidden, int64_t hidden_stride,
     // a warp per window; 4 CTAs of 128 threads fit an SM at 128 registers
     const long long ctas = (n_pooled_rows + kPoolWarps - 1) / kPoolWarps, cap = (long long)di.sm_count * 4;
     const int grid = (int)(ctas < cap ? ctas : cap);
-    posterior_pool_kernel<<<grid, kPoolThreads, sizeof(float) * kPoolWarps * pool_frames,
-                            static_cast<cudaStream_t>(stream)>>>(p);
+    // per-warp log weights of a window: above 48 KB (pool_frames > 3072)
+    // the kernel needs the opt-in shared memory limit
+    const size_t smem = sizeof(float) * kPoolWarps * (size_t)pool_frames;
+    if (smem > 48 * 1024 &&
+        !nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(posterior_pool_kernel), dev, di.smem_optin))
+        return NLE_ERR_CUDA;
+    posterior_pool_kernel<<<grid, kPoolThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
 }

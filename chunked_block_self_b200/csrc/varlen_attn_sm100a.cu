@@ -558,9 +558,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// Per device: dynamic smem opted in so far.
-int g_smem_set[64] = {};
-
 } // namespace
 
 extern "C" int nle_varlen_attn_fwd_ex(const void *q, const void *k, const void *v, void *out,
@@ -635,13 +632,8 @@ extern "C" int nle_varlen_attn_fwd_ex(const void *q, const void *k, const void *
         !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, stride, 64, kKeys))
         return NLE_ERR_CUDA;
 
-    const int slot = dev < 64 ? dev : 0;
-    if (dev >= 64 || g_smem_set[slot] < (int)smem) {
-        if (cudaFuncSetAttribute(reinterpret_cast<const void *>(varlen_attn_kernel),
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return NLE_ERR_CUDA;
-        g_smem_set[slot] = (int)smem;
-    }
+    if (!nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(varlen_attn_kernel), dev, di.smem_optin))
+        return NLE_ERR_CUDA;
     const int grid = (int)grid_ll;
     varlen_attn_kernel<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;

@@ -331,7 +331,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 using WKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, WParams);
-int g_smem_set[3][64] = {};
 
 } // namespace
 
@@ -406,13 +405,8 @@ extern "C" int nle_window_xattn_fwd_ex(const void *q, const void *k, const void 
         return NLE_ERR_CUDA;
 
     WKernel kern = KT == 1 ? window_xattn_kernel<1> : window_xattn_kernel<2>;
-    int &set = g_smem_set[KT][dev < 64 ? dev : 0];
-    if (dev >= 64 || set < (int)smem) {
-        if (cudaFuncSetAttribute(reinterpret_cast<const void *>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return NLE_ERR_CUDA;
-        set = (int)smem;
-    }
+    if (!nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(kern), dev, di.smem_optin))
+        return NLE_ERR_CUDA;
     const long long max_windows = (long long)n_seq + total_frames / window_frames;
     const int grid = (int)(max_windows < di.sm_count ? max_windows : di.sm_count);
     kern<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tk, tv, tq, p);

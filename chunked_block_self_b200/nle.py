@@ -38,7 +38,8 @@ _i32p = ctypes.POINTER(ctypes.c_int32)
 class PathBuffers(ctypes.Structure):
     """nle_path_buffers: host tensors, then their device copies."""
     _fields_ = [(n, _vp) for n in ("q", "k", "v", "out", "qw", "kw", "vw", "out_w", "cu",
-                                    "d_q", "d_k", "d_v", "d_out", "d_qw", "d_kw", "d_vw", "d_out_w", "d_cu")]
+                                    "d_q", "d_k", "d_v", "d_out", "d_qw", "d_kw", "d_vw", "d_out_w", "d_cu",
+                                    "d_status")]
 
 
 _SIGS = {
@@ -324,11 +325,13 @@ _PATH_NAMES = ("q", "k", "v", "out", "qw", "kw", "vw", "out_w")
 
 
 def nle_path_fwd_host(host: dict, dev: dict, block_frames: int = 200, window_frames: int = 15,
-                      queries_per_window: int = 3, n_chunks: int = 0, stream=None) -> None:
+                      queries_per_window: int = 3, n_chunks: int = 0, stream=None, dev_status=None) -> None:
     """Both kernels from host memory (nle_path_fwd_host).  ``host`` and ``dev``
     map q, k, v, out, qw, kw, vw, out_w to bf16 [rows, heads, 64] tensors on the
     CPU (pinned for overlap) and on the GPU, and cu to int32 [n_seq + 1].
-    Returns once the work is queued on ``stream``."""
+    ``dev_status`` (optional CUDA int32 [1]) receives the first in-kernel
+    error (a wait that ran out).  Returns once the work is queued on
+    ``stream``."""
     for name in _PATH_NAMES:
         h, d = host[name], dev[name]
         if h.device.type != "cpu" or h.dtype != torch.bfloat16 or not h.is_contiguous():
@@ -340,8 +343,11 @@ def nle_path_fwd_host(host: dict, dev: dict, block_frames: int = 200, window_fra
     if hcu.device.type != "cpu" or hcu.dtype != torch.int32 or not hcu.is_contiguous():
         raise ValueError("host cu: contiguous CPU int32 tensor required")
     _dev_tensor(dcu, "dev cu", torch.int32)
+    if dev_status is not None:
+        _dev_tensor(dev_status, "dev_status", torch.int32)
     b = PathBuffers(*[host[n].data_ptr() for n in _PATH_NAMES], hcu.data_ptr(),
-                    *[dev[n].data_ptr() for n in _PATH_NAMES], dcu.data_ptr())
+                    *[dev[n].data_ptr() for n in _PATH_NAMES], dcu.data_ptr(),
+                    dev_status.data_ptr() if dev_status is not None else None)
     heads = host["q"].shape[1]
     _check(_lib.nle_path_fwd_host(ctypes.byref(b), hcu.numel() - 1, host["q"].shape[0], host["qw"].shape[0],
                                   heads, host["q"].shape[2], block_frames, window_frames, queries_per_window,

@@ -26,10 +26,13 @@
  * Conventions for every attention entry point below (the pooling and CTC
  * entry points state their own layouts):
  *  - Tensor pointers (q, k, v, out, cu_seqlens, dev_status) are DEVICE
- *    pointers owned by the caller.  The library never allocates, frees or
- *    synchronises; every launch is asynchronous on `stream` (a cudaStream_t;
- *    NULL = the legacy default stream).  Host-side table functions take HOST
- *    pointers and say so.
+ *    pointers owned by the caller.  The kernel entry points never allocate,
+ *    free or synchronise; every launch is asynchronous on `stream` (a
+ *    cudaStream_t; NULL = the legacy default stream).  Host-side table
+ *    functions take HOST pointers and say so.  The one exception is
+ *    nle_path_fwd_host, which creates two streams and three events per
+ *    device on its first call (kept for the life of the process) and whose
+ *    copies block the calling thread unless the host buffers are pinned.
  *  - q, k, v, out hold bf16 values, row-major [rows][heads][d_head]: one row
  *    per frame (or per query), heads next, d_head contiguous.  d_head must be
  *    64.  Base pointers must be 16-byte aligned.
@@ -62,7 +65,7 @@
 extern "C" {
 #endif
 
-#define NLE_ABI_VERSION 1
+#define NLE_ABI_VERSION 2
 
 typedef enum {
     NLE_OK = 0,
@@ -260,6 +263,12 @@ int nle_posterior_pool_fwd(const void *hidden, int64_t hidden_stride, int dim, c
  *   cu                  int32 [n_seq + 1], non-decreasing from 0
  * Device buffers, owned by the caller, of the same shapes: d_q ... d_cu.
  *
+ * Resources: on its first call on a device this entry point creates two
+ * non-blocking streams and three events for that device, kept until the
+ * process exits (it allocates no memory).  The host buffers should be
+ * page-locked (cudaHostAlloc / cudaHostRegister): with pageable memory the
+ * copies are staged by the driver and block the calling thread.
+ *
  * The utterances are split into n_chunks chunks of consecutive utterances
  * (0 selects 8; at most n_seq).  For each chunk the input rows are copied to
  * the device, both kernels run on the chunk (each kernel call takes the
@@ -281,6 +290,12 @@ typedef struct {
     const int32_t *cu;         /* host cu_seqlens                           */
     void *d_q, *d_k, *d_v, *d_out, *d_qw, *d_kw, *d_vw, *d_out_w;
     int32_t *d_cu;             /* device copies (caller-owned)              */
+    int32_t *d_status;         /* nullable device int32: receives the first
+                                  in-kernel error of either kernel (a wait
+                                  that ran out: NLE_ERR_TIMEOUT); never
+                                  reset by the library.  With NULL such an
+                                  error goes unreported and the rows of the
+                                  work item concerned are left unwritten.  */
 } nle_path_buffers;
 
 int nle_path_fwd_host(const nle_path_buffers *b, int n_seq, int64_t total_frames, int64_t n_query_rows,

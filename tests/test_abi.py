@@ -27,7 +27,7 @@ def test_header_declarations_are_exported():
 
 
 def test_version_and_status_strings():
-    assert nle.nle_version() == 1
+    assert nle.nle_version() == 2
     for code in (0, -1, -2, -3, -4, -5):
         assert nle.nle_status_string(code).startswith("NLE_")
     assert nle.nle_status_string(-99) == "unknown nle status"

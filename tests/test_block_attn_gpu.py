@@ -107,6 +107,31 @@ def test_config_full_size_sampled(cfg, cuda_device):
     assert torch.isfinite(out.float()).all()
 
 
+def _per_item_rel_l2(got, ref, cu, B):
+    """Largest relative L2 error of any single (block, head) item."""
+    seq, j, start, ln = oracle.block_table(cu, B)
+    g = got.float().cpu().double().numpy()
+    worst = 0.0
+    for s0, n in zip(start.tolist(), ln.tolist()):
+        e = np.linalg.norm(g[s0:s0 + n] - ref[s0:s0 + n], axis=(0, 2))
+        r = np.maximum(np.linalg.norm(ref[s0:s0 + n], axis=(0, 2)), 1e-30)
+        worst = max(worst, float((e / r).max()))
+    return worst
+
+
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_config_full_size_every_output(cfg, cuda_device):
+    """Configs 3 (16 long utterances) and 4 (batch of 128) at full size:
+    every output of the launch against the oracle, as one tensor within the
+    tolerance, and item by item (every (block, head) within twice it), so a
+    single corrupted item among thousands cannot hide in the average."""
+    x = wl.block_inputs(cfg)
+    out = _run(x, cuda_device)
+    ref = oracle.block_attn(x["q"], x["k"], x["v"], x["cu"], block_frames=200)
+    _compare(out, ref)
+    assert _per_item_rel_l2(out, ref, x["cu"], 200) <= 2 * REL_L2
+
+
 def test_block_locality_bit_exact(cuda_device):
     x = wl.block_inputs(lengths=[530, 90], heads=4, seed=31)
     out = _run(x, cuda_device)

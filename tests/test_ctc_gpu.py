@@ -91,6 +91,33 @@ def test_full_size_sampled(cuda_device):
     torch.cuda.empty_cache()
 
 
+def test_full_size_every_frame_and_token(cuda_device):
+    """The batch-128 workload at full size (58,903 frames x 100,353 classes,
+    11.8 GB of bf16 logits generated on the device): the class of every
+    frame and the token stream of every utterance, bit for bit against the
+    oracle (which reads the logits in slices of 2,048 frames copied to the
+    host and decodes its own classes)."""
+    nle = _nle()
+    lengths = wl.draw_lengths(4)
+    cu_h = wl.cu_seqlens(lengths)
+    cu = torch.from_numpy(cu_h).to(cuda_device)
+    logits = wl.ctc_logits(lengths, seed=4004, device=cuda_device)
+    fc, tok, nt = nle.ctc_greedy(logits, cu)
+    torch.cuda.synchronize()
+    T = logits.shape[0]
+    ref_cls = np.empty(T, np.int64)
+    for a in range(0, T, 2048):
+        ref_cls[a:a + 2048] = oracle.ctc_frame_classes(logits[a:a + 2048].cpu())
+    del logits
+    torch.cuda.empty_cache()
+    np.testing.assert_array_equal(fc.cpu().numpy(), ref_cls)
+    ref_tok = oracle.ctc_collapse(ref_cls, cu_h)
+    tok, nt = tok.cpu().numpy(), nt.cpu().numpy()
+    for u in range(len(lengths)):
+        assert nt[u] == len(ref_tok[u])
+        assert tok[cu_h[u]:cu_h[u] + nt[u]].tolist() == ref_tok[u]
+
+
 def test_invalid_offsets_give_zero_tokens(cuda_device):
     lengths = [10, 10]
     logits = wl.ctc_logits(lengths, n_classes=9, seed=6)

@@ -42,8 +42,11 @@ def test_host_path_equals_device_path(chunks, pinned, cuda_device):
     dev = {n: torch.empty(t.shape, dtype=t.dtype, device=cuda_device) for n, t in host.items()}
     host["out"].fill_(float("nan"))
     host["out_w"].fill_(float("nan"))
-    nle.nle_path_fwd_host(host, dev, block_frames=B, window_frames=W, queries_per_window=QW, n_chunks=chunks)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    nle.nle_path_fwd_host(host, dev, block_frames=B, window_frames=W, queries_per_window=QW, n_chunks=chunks,
+                          dev_status=status)
     torch.cuda.current_stream().synchronize()
+    assert int(status.item()) == 0
     assert torch.equal(host["out"], ref)
     assert torch.equal(host["out_w"], ref_w)
 

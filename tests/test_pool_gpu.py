@@ -167,3 +167,30 @@ def test_full_size_sampled(cuda_device):
     _compare(np.array(got), np.array(ref))
     rw = oracle.blank_weights(x["logits"][:2000].cpu())
     np.testing.assert_allclose(w[:2000].cpu().double().numpy(), rw, rtol=1e-5, atol=1e-6)
+
+
+def test_full_size_every_row(cuda_device):
+    """Batch-128 workload at full size (58,903 frames x 1024, 256 mid-layer
+    classes, windows of 2), generated on the device: every pooled row and
+    every weight against the oracle."""
+    nle = _nle()
+    lengths = wl.draw_lengths(4)
+    cu = wl.cu_seqlens(lengths)
+    x = wl.pool_inputs(lengths, seed=77, device=cuda_device)
+    cu_d = torch.from_numpy(cu).to(cuda_device)
+    n_rows = int(oracle.pooled_rows(cu, 2)[-1])
+    pooled, w = nle.posterior_pool(x["hidden"], x["logits"], cu_d, 2, n_rows=n_rows)
+    torch.cuda.synchronize()
+    ref, rw = oracle.posterior_pool(x["hidden"].cpu(), x["logits"].cpu(), cu, 2)
+    _compare(pooled.float().cpu().double().numpy(), ref)
+    np.testing.assert_allclose(w.cpu().double().numpy(), rw, rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("P", [3072, 3073, 4096])
+def test_largest_pool_windows(P, cuda_device):
+    """Windows of up to 4096 frames (the documented maximum), whose per-warp
+    weight buffers need more than the default 48 KB of shared memory."""
+    lengths = [2 * P + 5, P, 17]
+    cu = wl.cu_seqlens(lengths)
+    x = wl.pool_inputs(lengths, 64, 37, seed=P)
+    _check(x, cu, cuda_device, P, 64, 37)

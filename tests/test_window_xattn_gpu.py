@@ -75,6 +75,23 @@ def test_config5_full_size_sampled(cuda_device):
     assert torch.isfinite(out.float()).all()
 
 
+def test_config5_full_size_every_output(cuda_device):
+    """Config 5 (64 utterances of 4700 frames, 20,096 windows, 16 heads) at
+    full size: every query row of the launch against the oracle, as one
+    tensor within the tolerance and window by window (every (window, head)
+    within twice it)."""
+    cu = wl.cu_seqlens(wl.draw_lengths(5))
+    nq = 3 * len(oracle.window_table(cu, 15, 3)[0])
+    x = wl.window_inputs(nq, cfg=5)
+    out = _run(x, cuda_device)
+    ref = oracle.window_xattn(x["q"], x["k"], x["v"], x["cu"], 15, 3)
+    _compare(out, ref)
+    g = out.float().cpu().double().numpy().reshape(nq // 3, 3, 16, 64)
+    r = ref.reshape(nq // 3, 3, 16, 64)
+    e = np.linalg.norm(g - r, axis=(1, 3)) / np.maximum(np.linalg.norm(r, axis=(1, 3)), 1e-30)
+    assert e.max() <= 2 * REL_L2, f"worst window rel_l2={e.max():.3e}"
+
+
 def test_window_locality_bit_exact(cuda_device):
     x = _inputs([47, 15], 4, seed=41)
     out = _run(x, cuda_device)

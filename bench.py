@@ -2,22 +2,28 @@
 cross-attention over one packed batch per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nle|reference]
+                    [--config 1..5] [--seed S]
 
-A step is one pass of the whole path over the batch-128 workload (128
-utterances of 100-800 frames, 16 heads x 64, the model card's batch-128
-throughput setting): the 200-frame block self-attention of the encoder and
-the projector's 15-frame / 3-query windowed cross-attention over the same
-utterances.  Inputs are synthetic (seeded N(0,1) bf16), resident in HBM
-before timing; they total ~0.75 GB, larger than the 126 MB L2, so L2 is not
-flushed between steps.  One JSON line is printed by rank 0.
+A step is one pass of the whole path over one packed batch: the 200-frame
+block self-attention of the encoder and the projector's 15-frame / 3-query
+windowed cross-attention over the same utterances.  The default workload is
+config 4, the batch-128 one (128 utterances of 100-800 frames, 16 heads x
+64, the model card's batch-128 throughput setting); --config selects another
+of the five synthetic workloads.  Inputs are seeded N(0,1) bf16, resident in
+HBM before timing; each kernel is also timed alone (median over the K
+steps).  One JSON line is printed by rank 0.
+
+The `configs` field of the line times the kernels on all five workloads
+(median of >= 50 launches each, L2 flushed by a 256 MB write before every
+launch, and back to back for the two small workloads that fit in L2).
 
 Multi-GPU (torchrun, one process per GPU): data-parallel replicas, each
 rank runs its own batch of the same shape (weak scaling); there is no
 collective on the data path.  Time is the max over ranks.
 
 --impl reference times the fp64 CPU oracle (the test oracle, untuned) on the
-host cores for the same metric: each step is a bounded sample of (block,
-head) / (window, head) items of the same workload.
+host cores for the same metric: each step is a bounded sample of whole
+utterances of the same workload.
 """
 from __future__ import annotations
 
@@ -39,7 +45,8 @@ sys.path.insert(0, ROOT)
 from chunked_block_self_b200 import workloads as wl  # noqa: E402
 
 METRIC = "block-attn TFLOP/s & encoder frames/s on 1 B200; % of dense BF16 peak"
-CFG = 4
+CFG = 4          # the headline workload; --config changes it
+SEED = None      # --seed; None: the config's default seed
 B, W, QW, D = 200, 15, 3, 64
 
 # ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of each
@@ -50,14 +57,18 @@ B, W, QW, D = 200, 15, 3, 64
 NCU_TRAFFIC = {
     "block_attn": {"files": ("block_attn_sm100a.cu", "attn_softmax.cuh", "nle_device.cuh"),
                    "source_sha256": "2e6ebd9f63407760f95d35cad80618ba9226f66a254b7f3478e5c0a62b707595",
-                   "traffic_over_algorithmic": (377232640 + 66526720) / 482533376},
+                   "traffic_over_algorithmic": (377232640 + 66526720) / 482533376,
+                   "tensor_pipe_pct": 19.2},
     "window_xattn": {"files": ("window_xattn_sm100a.cu", "nle_device.cuh"),
                      "source_sha256": "43ecd044325aac9d122bc38ba666274726781c3720caf2f2a5fcb5b34fb21737",
                      "traffic_over_algorithmic": (265946112 + 7618304) / 290320384},
     # full-utterance attention: the long-clip workload, the same launch as the bench's
     "varlen_attn": {"files": ("varlen_attn_sm100a.cu", "attn_softmax.cuh", "nle_device.cuh"),
                     "source_sha256": "f97abe68c26d62ac374fa754a2f1b1536b5e4cc4598e43d5712680b93a44f41f",
-                    "traffic_over_algorithmic": (343228160 + 91153152) / 439304192},
+                    "traffic_over_algorithmic": (343228160 + 91153152) / 439304192,
+                    "tensor_pipe_pct": 25.6},
+    "qkv_attn": {"files": ("qkv_attn_sm100a.cu", "attn_softmax.cuh", "nle_device.cuh"),
+                 "source_sha256": "", "traffic_over_algorithmic": None},
     # CTC argmax: captured on 16 utterances (3,300 rows, 662.4 MB); traffic grows
     # with rows, so the ratio is applied to the full batch
     "ctc_argmax": {"files": ("ctc_sm100a.cu", "nle_device.cuh"),
@@ -79,6 +90,16 @@ def ncu_traffic(kernel: str, algorithmic_bytes: int):
     if e["source_sha256"] != kernel_source_sha(kernel):
         return None
     return e["traffic_over_algorithmic"] * algorithmic_bytes
+
+
+def ncu_tensor_pipe_pct(kernel: str):
+    """sm__pipe_tensor_cycles_active (% of active cycles) from the ncu capture
+    of `kernel`, or None when the source changed since (or none was taken).
+    It counts the padded MMA work (keys up to ceil16(L), 128-row tiles)."""
+    e = NCU_TRAFFIC.get(kernel)
+    if not e or "tensor_pipe_pct" not in e or e["source_sha256"] != kernel_source_sha(kernel):
+        return None
+    return e["tensor_pipe_pct"]
 
 
 def measured_peaks():
@@ -238,22 +259,44 @@ def cpu_info():
 
 
 # ------------------------------------------------------------------ arms
+WORKLOAD_NAMES = {
+    1: "single utterance: 400 frames (8 s at 50 Hz), 8 heads x 64",
+    2: "800-frame bucket: one utterance of 800 frames (16 s), 16 heads x 64, values x0.5",
+    3: "long clips: 16 utterances of 1950-4700 frames (39-94 s), partial last blocks, 16 heads x 64",
+    4: "batch-128: 128 utterances of 100-800 frames (2-16 s at 50 Hz), 16 heads x 64",
+    5: "projector batch: 64 utterances of 4700 frames (94 s), 16 heads x 64",
+}
+
+
+def base_seed(rank):
+    return (wl.default_seed(CFG) if SEED is None else SEED) + rank
+
+
 def build_inputs(rank):
-    seed = wl.default_seed(CFG) + rank
+    """Block inputs (host) of the headline workload and window inputs over the
+    same utterances; the projector workload's window inputs are those of
+    config 5."""
+    seed = base_seed(rank)
     x = wl.block_inputs(CFG, seed=seed)
     lengths, heads = x["lengths"], x["heads"]
     n_win = sum(-(-int(t) // W) for t in lengths)
-    y = wl.window_inputs(QW * n_win, cfg=None, lengths=lengths, heads=heads, seed=seed + 100)
+    if CFG == 5:
+        y = wl.window_inputs(QW * n_win, cfg=5, seed=seed)
+    else:
+        y = wl.window_inputs(QW * n_win, cfg=None, lengths=lengths, heads=heads, seed=seed + 100)
     return x, y
 
 
 def config_dict(x, n_win):
-    return {"workload": "batch-128: 128 utterances of 100-800 frames (2-16 s at 50 Hz), 16 heads x 64; "
-                        "200-frame block self-attention + 15-frame/3-query windowed cross-attention",
-            "n_seq": int(len(x["lengths"])), "total_frames": int(x["total"]), "heads": int(x["heads"]),
-            "d_head": D, "block_frames": B, "window_frames": W, "queries_per_window": QW,
-            "windows": int(n_win), "seed": wl.default_seed(CFG),
-            "l2": "inputs ~0.75 GB per rank > 126 MB L2; not flushed between steps",
+    gb = (4 * x["q"].numel() * 2 + (2 * QW * n_win + 2 * int(x["total"])) * int(x["heads"]) * D * 2) / 1e9
+    l2 = (f"inputs ~{gb:.2f} GB per rank > 126 MB L2; not flushed between steps" if gb > 0.126 else
+          f"inputs ~{gb * 1e3:.0f} MB per rank fit in the 126 MB L2; back to back, hot (the `configs` "
+          "field also times them L2-flushed)")
+    return {"workload": f"config {CFG}, {WORKLOAD_NAMES[CFG]}; 200-frame block self-attention + "
+                        "15-frame/3-query windowed cross-attention over the same utterances",
+            "config": CFG, "n_seq": int(len(x["lengths"])), "total_frames": int(x["total"]),
+            "heads": int(x["heads"]), "d_head": D, "block_frames": B, "window_frames": W,
+            "queries_per_window": QW, "windows": int(n_win), "seed": base_seed(0), "l2": l2,
             "parallelism": "data-parallel replicas by utterance (no collective)"}
 
 
@@ -288,6 +331,151 @@ def run_reference(args, rank, world):
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def time_launches(fn, stream, reps, flush=None):
+    """Median and mean (ms) of `reps` launches of fn, each bracketed by CUDA
+    events on `stream`; with `flush`, a write of that buffer (larger than
+    L2) precedes every launch."""
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts), float(np.mean(ts))
+
+
+def measure_configs(nle, dev, stream, reps, rank, hbm_peak, tf_peak):
+    """Each kernel of the path on each of the five workloads, alone: the
+    block kernel on configs 1-4, the window kernel on configs 4 and 5 (the
+    projector batch: 64 x 4700 frames, 20,096 windows).  Inputs are drawn on
+    the device (seeded torch generator, same distributions as the host
+    recipe).  Median of `reps` launches with L2 flushed before each; the
+    two small workloads (which fit in L2) are also timed back to back."""
+    sp = stream.cuda_stream
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    for c in (1, 2, 3, 4, 5):
+        seed = wl.default_seed(c) + rank
+        lengths = wl.draw_lengths(c, seed)
+        heads = wl.CONFIGS[c].heads
+        total = int(sum(int(t) for t in lengths))
+        cu = torch.from_numpy(wl.cu_seqlens(lengths)).to(dev)
+        e = {"workload": WORKLOAD_NAMES[c], "n_seq": int(len(lengths)), "total_frames": total, "heads": heads,
+             "seed": seed, "reps": reps, "timing": "median of CUDA-event times of single launches"}
+        if c <= 4:
+            x = wl.block_inputs(c, seed=seed, device=dev)
+            out = torch.empty_like(x["q"])
+
+            def blk():
+                nle.nle_block_attn_fwd(x["q"], x["k"], x["v"], out, cu, len(lengths), total, heads, D, B,
+                                       stream=sp)
+
+            for _ in range(3):
+                blk()
+            f, by = block_work(lengths, heads)
+            med, mean = time_launches(blk, stream, reps, flush)
+            blk_e = {"us_flushed": 1e3 * med, "us_flushed_mean": 1e3 * mean,
+                     "tflops": f / (med * 1e-3) / 1e12, "gbs": by / (med * 1e-3) / 1e9,
+                     "pct_of_hbm_peak": 100.0 * by / (med * 1e-3) / 1e9 / hbm_peak,
+                     "pct_of_dense_bf16_peak": 100.0 * f / (med * 1e-3) / 1e12 / tf_peak,
+                     "frames_per_s": total / (med * 1e-3), "algorithmic_flops": f, "algorithmic_bytes": by,
+                     "hbm_floor_us": 1e6 * by / (hbm_peak * 1e9)}
+            if by < (96 << 20):   # fits in L2: the layer-after-layer case
+                hot, _ = time_launches(blk, stream, reps)
+                blk_e.update({"us_hot": 1e3 * hot, "tflops_hot": f / (hot * 1e-3) / 1e12,
+                              "frames_per_s_hot": total / (hot * 1e-3)})
+            if c == 2:   # the same call in each of the encoder's 16 layers
+                blk_e["frames_per_s_16_layer_stack_flushed"] = total / (16 * med * 1e-3)
+                blk_e["frames_per_s_16_layer_stack_hot"] = total / (16 * hot * 1e-3)
+            e["block_attn"] = blk_e
+            del x, out
+        if c >= 4:
+            n_win = sum(-(-int(t) // W) for t in lengths)
+            y = wl.window_inputs(QW * n_win, cfg=c, seed=seed, device=dev)
+            ow = torch.empty_like(y["q"])
+
+            def win():
+                nle.nle_window_xattn_fwd(y["q"], y["k"], y["v"], ow, cu, len(lengths), total, QW * n_win, heads,
+                                         D, W, QW, stream=sp)
+
+            for _ in range(3):
+                win()
+            f, by, _ = window_work(lengths, heads)
+            med, mean = time_launches(win, stream, reps, flush)
+            e["window_xattn"] = {"windows": int(n_win), "us_flushed": 1e3 * med, "us_flushed_mean": 1e3 * mean,
+                                 "gbs": by / (med * 1e-3) / 1e9,
+                                 "pct_of_hbm_peak": 100.0 * by / (med * 1e-3) / 1e9 / hbm_peak,
+                                 "tflops": f / (med * 1e-3) / 1e12, "algorithmic_bytes": by,
+                                 "hbm_floor_us": 1e6 * by / (hbm_peak * 1e9)}
+            del y, ow
+        res[str(c)] = e
+        torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_qkv_attn(nle, dev, stream, reps, rank, lengths, tf_peak):
+    """The QKV projection fused with block attention on the step's
+    utterances at the encoder's width (d_model 1024 = 16 heads x 64): X
+    N(0, 1), W N(0, 1/1024), bias N(0, 0.25), all bf16, drawn on the device.
+    Median of `reps` launches, L2 flushed before each.  The same work done
+    unfused -- the projection as one cuBLAS GEMM (torch) writing Q|K|V to
+    memory, then the block kernel reading them -- is timed beside it."""
+    sp = stream.cuda_stream
+    heads, dm = 16, 1024
+    cu_h = wl.cu_seqlens(lengths)
+    T = int(cu_h[-1])
+    cu = torch.from_numpy(cu_h).to(dev)
+    seed = wl.default_seed(CFG) + 5000 + rank
+    x = wl.device_normal((T, dm), 1.0, seed, dev)
+    w = wl.device_normal((3 * heads * 64, dm), 1.0 / 32.0, seed + 1, dev)
+    b = wl.device_normal((3 * heads * 64,), 0.5, seed + 2, dev)
+    out = torch.empty((T, heads, 64), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def fused():
+        nle.nle_block_attn_qkv_fwd(x, w, b, out, cu, block_frames=B, stream=sp)
+
+    qkv = torch.empty((T, 3 * heads * 64), dtype=torch.bfloat16, device=dev)
+    out2 = torch.empty_like(out)
+
+    def unfused():
+        torch.addmm(b, x, w.t(), out=qkv)
+        q3 = qkv.view(T, 3, heads, 64)
+        nle.nle_block_attn_fwd_ex(q3[:, 0], q3[:, 1], q3[:, 2], out2, cu, len(lengths), T, heads, D, B,
+                                  row_stride_qkv=3 * heads * 64, stream=sp)
+
+    for _ in range(3):
+        fused()
+        unfused()
+    med, mean = time_launches(fused, stream, reps, flush)
+    umed, _ = time_launches(unfused, stream, reps, flush)
+    f_att, _ = block_work(lengths, heads)
+    f_proj = 2 * T * dm * 3 * heads * 64
+    flops = f_proj + f_att
+    tflops = flops / (med * 1e-3) / 1e12
+    byt = 2 * (T * dm + 3 * heads * 64 * dm + 3 * heads * 64 + T * heads * 64)   # X, W, b read; O written
+    res = {"workload": f"config {CFG} utterances ({len(lengths)}, {T} frames), d_model {dm}, {heads} heads x 64, "
+                       "synthetic X ~ N(0,1), W ~ N(0,1/1024), bias ~ N(0,0.25), bf16",
+           "ms": med, "ms_mean": mean, "timing": f"median of {reps} launches, L2 flushed (256 MB write) before each",
+           "algorithmic_flops": flops, "projection_flops": f_proj, "attention_flops": f_att,
+           "tflops": tflops, "pct_of_dense_bf16_peak": 100.0 * tflops / tf_peak,
+           "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_peak, "unit": "TFLOP/s",
+                        "frac": tflops / tf_peak, "ai_flop_per_byte": flops / byt},
+           "tensor_pipe_pct": ncu_tensor_pipe_pct("qkv_attn"),
+           "unfused_ms": umed, "unfused_tflops": flops / (umed * 1e-3) / 1e12,
+           "unfused": "torch.addmm (cuBLAS) X W^T + b -> Q|K|V in memory, then the block kernel",
+           "speedup_vs_unfused": umed / med, "kernels": 1}
+    del x, w, b, out, qkv, out2, flush
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_nle(args, rank, world, local):
@@ -345,8 +533,9 @@ def run_nle(args, rank, world, local):
         barrier(world)
         torch.cuda.synchronize()
     elapsed_ms = start.elapsed_time(end)
-    t_blk = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)) / K
-    t_win = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(K)) / K
+    blk_ts = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K)]
+    win_ts = [ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(K)]
+    t_blk, t_win = statistics.median(blk_ts), statistics.median(win_ts)
     elapsed_ms = max_over_ranks(elapsed_ms, world)
     ms_step = elapsed_ms / K
 
@@ -409,16 +598,7 @@ def run_nle(args, rank, world, local):
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
         def timed(fn, reps):
-            ts = []
-            for _ in range(reps):
-                flush.fill_(1)
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fn()
-                b.record(stream)
-                torch.cuda.synchronize()
-                ts.append(a.elapsed_time(b))
-            return float(np.mean(ts))
+            return time_launches(fn, stream, reps, flush)[0]   # median
 
         px = wl.pool_inputs(clen, seed=wl.default_seed(CFG) + 4000 + rank, device=dev)
         pooled = torch.empty((n_rows, wl.HIDDEN_DIM), dtype=torch.bfloat16, device=dev)
@@ -429,12 +609,13 @@ def run_nle(args, rank, world, local):
 
         for _ in range(3):
             pool_step()
-        pool_ms = timed(pool_step, 20)
+        pool_ms = timed(pool_step, 50)
         # hidden and logits once, pooled rows and weights written
         pool_bytes = n_fr * (wl.HIDDEN_DIM + wl.CHAR_CLASSES) * 2 + n_rows * wl.HIDDEN_DIM * 2 + n_fr * 4
         pool = {"frames": n_fr, "rows": n_rows, "pool_frames": wl.POOL_FRAMES, "dim": wl.HIDDEN_DIM,
                 "char_classes": wl.CHAR_CLASSES, "ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
-                "algorithmic_bytes": pool_bytes, "l2": "flushed (256 MB write) before each launch", "kernels": 1}
+                "algorithmic_bytes": pool_bytes, "l2": "flushed (256 MB write) before each launch", "kernels": 1,
+                "timing": "median of 50 launches"}
         del px, pooled, pw
 
         logits = wl.ctc_logits(rows_u, seed=wl.default_seed(CFG) + 3000 + rank, device=dev)
@@ -447,13 +628,14 @@ def run_nle(args, rank, world, local):
 
         for _ in range(3):
             ctc_step()
-        ctc_ms = timed(ctc_step, 10)
+        ctc_ms = timed(ctc_step, 20)
         # logits once; frame classes written, read twice by the collapse;
         # tokens written; one count per utterance
         ctc_bytes = logits.numel() * 2 + n_rows * 12 + len(clen) * 4
         ctc = {"rows": n_rows, "utterances": len(clen), "classes": int(logits.shape[1]), "ms": ctc_ms,
                "rows_per_s": n_rows / (ctc_ms * 1e-3), "gbs": ctc_bytes / (ctc_ms * 1e-3) / 1e9,
                "algorithmic_bytes": ctc_bytes, "l2": "flushed (256 MB write) before each launch", "kernels": 2,
+               "timing": "median of 20 launches",
                # the argmax kernel's DRAM bytes (logits once, classes written)
                "traffic_argmax": ncu_traffic("ctc_argmax", logits.numel() * 2 + n_rows * 4)}
         del logits, flush
@@ -475,14 +657,7 @@ def run_nle(args, rank, world, local):
         for _ in range(3):
             va_step()
         torch.cuda.synchronize()
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        kv_reps = 20
-        a0.record(stream)
-        for _ in range(kv_reps):
-            va_step()
-        a1.record(stream)
-        torch.cuda.synchronize()
-        va_ms = a0.elapsed_time(a1) / kv_reps
+        va_ms, _ = time_launches(va_step, stream, 50)   # median; inputs > L2
         lens_v = [int(t) for t in xv["lengths"]]
         hv_ = int(xv["heads"])
         va_flops = 4 * D * hv_ * sum(t * t for t in lens_v)
@@ -492,10 +667,17 @@ def run_nle(args, rank, world, local):
               "frames": int(sum(lens_v)), "ms": va_ms, "tflops": va_flops / (va_ms * 1e-3) / 1e12,
               "algorithmic_flops": va_flops, "algorithmic_bytes": va_bytes,
               "l2": "inputs ~0.32 GB > 126 MB L2; not flushed", "kernels": 1,
+              "timing": "median of 50 launches", "tensor_pipe_pct": ncu_tensor_pipe_pct("varlen_attn"),
               "traffic": ncu_traffic("varlen_attn", va_bytes)}
         del qv, kv, vv, outv
 
     hbm_peak, tf_peak, tf_sust, peak_src = measured_peaks()
+    per_cfg = None
+    if not args.no_configs:
+        per_cfg = measure_configs(nle, dev, stream, args.config_reps, rank, hbm_peak, tf_peak)
+    qkv_att = None
+    if not args.no_qkv:
+        qkv_att = measure_qkv_attn(nle, dev, stream, args.config_reps, rank, lengths, tf_peak)
     if va is not None:
         va["pct_of_dense_bf16_peak"] = 100.0 * va["tflops"] / tf_peak
         va["roofline"] = {"bound": "tensor", "achieved": va["tflops"], "peak": tf_peak, "unit": "TFLOP/s",
@@ -515,10 +697,18 @@ def run_nle(args, rank, world, local):
         "frames_per_s": world * frames_step / (ms_step * 1e-3),
         "pct_of_dense_bf16_peak": 100.0 * value / (world * tf_peak),
         "block_attn": {"tflops": blk_tflops, "pct_of_dense_bf16_peak": 100.0 * blk_tflops / tf_peak,
-                       "achieved_gbs": achieved_gbs, "ms": t_blk, "frames_per_s": frames_step / (t_blk * 1e-3),
+                       "achieved_gbs": achieved_gbs, "ms": t_blk, "ms_mean": float(np.mean(blk_ts)),
+                       "timing": f"median of {K} launches (CUDA events around each)",
+                       "frames_per_s": frames_step / (t_blk * 1e-3),
+                       "frames_per_s_16_layer_stack": frames_step / (16 * t_blk * 1e-3),
                        "attainable_tflops": min(tf_peak, f_blk / by_blk * hbm_peak / 1e3),
-                       "ai_flop_per_byte": f_blk / by_blk},
-        "window_xattn": {"gbs": by_win / (t_win * 1e-3) / 1e9, "ms": t_win, "tflops": f_win / (t_win * 1e-3) / 1e12,
+                       "ai_flop_per_byte": f_blk / by_blk,
+                       "tensor_pipe_pct": ncu_tensor_pipe_pct("block_attn")},
+        "tensor_pipe_pct": ncu_tensor_pipe_pct("block_attn"),
+        "qkv_attn": qkv_att,
+        "configs": per_cfg,
+        "window_xattn": {"gbs": by_win / (t_win * 1e-3) / 1e9, "ms": t_win, "ms_mean": float(np.mean(win_ts)),
+                         "tflops": f_win / (t_win * 1e-3) / 1e12,
                          "pct_of_hbm_peak": 100.0 * by_win / (t_win * 1e-3) / 1e9 / hbm_peak,
                          "algorithmic_bytes": by_win, "traffic": ncu_traffic("window_xattn", by_win)},
         "roofline": {"kernel": "block_attn_kernel", "bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
@@ -551,9 +741,17 @@ def main():
     ap.add_argument("--no-varlen", action="store_true", help="skip the full-utterance attention measurement")
     ap.add_argument("--ctc-utts", type=int, default=0,
                     help="pool and decode only the first N utterances (0: the whole batch)")
+    ap.add_argument("--config", type=int, choices=[1, 2, 3, 4, 5], default=4,
+                    help="the step's workload (default 4, the batch-128 one)")
+    ap.add_argument("--seed", type=int, default=None, help="input seed (default: 1000 + config)")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel timings")
+    ap.add_argument("--no-qkv", action="store_true", help="skip the fused QKV projection + attention timing")
+    ap.add_argument("--config-reps", type=int, default=50, help="launches per kernel and config (>= 50)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    global CFG, SEED
+    CFG, SEED = args.config, args.seed
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", "1"))

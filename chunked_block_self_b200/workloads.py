@@ -96,10 +96,11 @@ def bf16_normal(rng: np.random.Generator, shape, factor: float = 1.0) -> torch.T
 
 def block_inputs(cfg: int | None = None, seed: int | None = None, *, lengths=None,
                  heads: int | None = None, d_head: int = 64, factor: float | None = None,
-                 block_frames: int | None = None) -> dict:
+                 block_frames: int | None = None, device=None) -> dict:
     """Q, K, V (bf16 CPU, [total_frames, heads, d_head]) plus offsets.
 
     Either a config number, or explicit ``lengths``/``heads`` for custom cases.
+    With ``device``, Q, K and V are drawn there instead (see device_normal).
     """
     if cfg is not None:
         w = CONFIGS[cfg]
@@ -114,9 +115,14 @@ def block_inputs(cfg: int | None = None, seed: int | None = None, *, lengths=Non
     heads = 1 if heads is None else heads
     factor = 1.0 if factor is None else factor
     block_frames = 200 if block_frames is None else block_frames
-    rng = np.random.default_rng(12345 if seed is None else seed + 7)
     cu = cu_seqlens(lengths)
     total = int(cu[-1])
+    if device is not None:
+        s0 = 12345 if seed is None else seed + 7
+        q, k, v = (device_normal((total, heads, d_head), factor, s0 + i, device) for i in range(3))
+        return dict(q=q, k=k, v=v, cu=cu, lengths=lengths, heads=heads, d_head=d_head,
+                    block_frames=block_frames, total=total)
+    rng = np.random.default_rng(12345 if seed is None else seed + 7)
     q = bf16_normal(rng, (total, heads, d_head), factor)
     k = bf16_normal(rng, (total, heads, d_head), factor)
     v = bf16_normal(rng, (total, heads, d_head), factor)
@@ -124,14 +130,27 @@ def block_inputs(cfg: int | None = None, seed: int | None = None, *, lengths=Non
                 block_frames=block_frames, total=total)
 
 
+def device_normal(shape, factor: float, seed: int, device) -> torch.Tensor:
+    """bf16 N(0,1) * factor drawn on ``device`` from a torch generator seeded
+    with ``seed`` (other values than the host generator, same distribution):
+    for benchmark inputs too large to draw on the host quickly."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if factor != 1.0:
+        x *= factor
+    return x.to(torch.bfloat16)
+
+
 def window_inputs(n_query_rows: int, cfg: int | None = 5, seed: int | None = None, *,
                   lengths=None, heads: int | None = None, d_head: int = 64,
-                  factor: float | None = None) -> dict:
+                  factor: float | None = None, device=None) -> dict:
     """Inputs of the windowed cross-attention.
 
     ``n_query_rows`` is the number of query rows the caller's window plan asks
     for (this module does not cut windows).  K and V are [total_frames, heads,
-    d_head]; Q is [n_query_rows, heads, d_head]; all bf16 CPU tensors.
+    d_head]; Q is [n_query_rows, heads, d_head]; bf16 CPU tensors, or tensors
+    drawn on ``device`` (see device_normal) when one is given.
     """
     w = CONFIGS[cfg] if cfg is not None else None
     if w is not None:
@@ -143,9 +162,15 @@ def window_inputs(n_query_rows: int, cfg: int | None = 5, seed: int | None = Non
     lengths = np.asarray(lengths, np.int64)
     heads = 1 if heads is None else heads
     factor = 1.0 if factor is None else factor
-    rng = np.random.default_rng(54321 if seed is None else seed + 11)
     cu = cu_seqlens(lengths)
     total = int(cu[-1])
+    if device is not None:
+        s0 = 54321 if seed is None else seed + 11
+        k = device_normal((total, heads, d_head), factor, s0, device)
+        v = device_normal((total, heads, d_head), factor, s0 + 1, device)
+        q = device_normal((int(n_query_rows), heads, d_head), factor, s0 + 2, device)
+        return dict(q=q, k=k, v=v, cu=cu, lengths=lengths, heads=heads, d_head=d_head, total=total)
+    rng = np.random.default_rng(54321 if seed is None else seed + 11)
     k = bf16_normal(rng, (total, heads, d_head), factor)
     v = bf16_normal(rng, (total, heads, d_head), factor)
     q = bf16_normal(rng, (int(n_query_rows), heads, d_head), factor)

@@ -132,4 +132,111 @@ __device__ __forceinline__ void rescale_p(uint32_t tS, int ncols, float f)
     }
 }
 
+// ------------------------------------------------------------ one-tile rows
+// Rare path of one segment (whole warp): S of the segment is still intact
+// in TMEM (its P has not been stored yet), so it is streamed again in
+// 16-column chunks: first its max, then m moves up by a whole k so that max
+// maps to <= 0, the segment's P is recomputed and stored, and the P already
+// written (columns < C0/2) are rescaled by 2^-k.  A chunk's P (columns
+// (C0+c)/2..+8) only overwrites S columns that have already been read.
+template <int W>
+__device__ __forceinline__ void softmax_rare(uint32_t tS, int C0, int L, float sl2, float &m, float &l)
+{
+    tmem_wait_ld();   // also completes a prefetch of the next segment
+    float mx = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < W; c += 16) {
+        uint32_t r[16];
+        tmem_ld16_nowait(tS + C0 + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            reg_fence(r[i]);
+            if (C0 + c + i < L)
+                mx = fmaxf(mx, __uint_as_float(r[i]));
+        }
+    }
+    const float y = mx * sl2 - m;
+    const int k = y > 0.f ? (int)ceilf(y) : 0;
+    const float f = k <= 126 ? __int_as_float((127 - k) << 23) : 0.f;
+    m += (float)k;
+    l *= f;
+#pragma unroll 1
+    for (int c = 0; c < W; c += 16) {
+        uint32_t r[16], pk[8];
+        tmem_ld16_nowait(tS + C0 + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            reg_fence(r[2 * i]);
+            reg_fence(r[2 * i + 1]);
+            const float a = C0 + c + 2 * i < L ? ex2_approx(fmaf(__uint_as_float(r[2 * i]), sl2, -m)) : 0.f;
+            const float b = C0 + c + 2 * i + 1 < L ? ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), sl2, -m)) : 0.f;
+            l += a + b;
+            pk[i] = pack_bf16x2(a, b);
+        }
+        tmem_st8p(tS + (C0 + c) / 2, pk);
+        tmem_wait_st();
+    }
+    if (C0 > 0)
+        rescale_p(tS, C0 / 2, f);
+}
+
+template <int NB, int SEG, int K>
+__device__ __forceinline__ void softmax_step(uint32_t tS, int L, float sl2, float &m, float &l, uint32_t (&cur)[SEG])
+{
+    constexpr int C0 = K * SEG;
+    constexpr int W = NB - C0 < SEG ? NB - C0 : SEG;
+    constexpr int C1 = C0 + SEG;
+    if (K > 0) {
+        seg_issue<W>(tS + C0, cur);
+        tmem_wait_ld();
+        seg_fence<W>(cur);
+    }
+    if (C0 + W > L)   // warp-uniform
+        seg_mask<W>(cur, C0, L);
+    uint32_t pk[W / 2];
+    float ymax;
+    const float ls = seg_exp<W>(cur, pk, sl2, m, ymax);
+    if (__any_sync(kFull, !(ymax <= kYMax))) {
+        softmax_rare<W>(tS, C0, L, sl2, m, l);
+    } else {
+        l += ls;
+        seg_store<W>(tS + C0 / 2, pk);
+    }
+    if constexpr (C1 < NB) {
+        if (L > C1)
+            softmax_step<NB, SEG, K + 1>(tS, L, sl2, m, l, cur);
+    }
+}
+
+// Softmax of a whole row tile whose keys fit one S of NB <= 256 columns
+// (the block kernels).  Returns this lane's row sum; P (bf16) is left over
+// the first NB/2 columns of S.  Segments wholly at or past L are skipped (the MMAs stop at
+// ceil16(L) keys).
+template <int NB, int SEG>
+__device__ __forceinline__ float block_softmax_rows(uint32_t tS, int L, float sl2)
+{
+    static_assert(SEG % 16 == 0 && SEG >= 16, "segments");
+    constexpr int W0 = NB < SEG ? NB : SEG;
+    uint32_t buf[SEG];
+    seg_issue<W0>(tS, buf);
+    tmem_wait_ld();
+    seg_fence<W0>(buf);
+    // first shift: max of the first 16 keys (keys >= L masked first)
+    if (W0 > L)
+        seg_mask<W0>(buf, 0, L);
+    float m = fmax3(fmax3(__uint_as_float(buf[0]), __uint_as_float(buf[1]), __uint_as_float(buf[2])),
+                    fmax3(__uint_as_float(buf[3]), __uint_as_float(buf[4]), __uint_as_float(buf[5])),
+                    fmax3(__uint_as_float(buf[6]), __uint_as_float(buf[7]), __uint_as_float(buf[8])));
+    m = fmax3(m, fmax3(__uint_as_float(buf[9]), __uint_as_float(buf[10]), __uint_as_float(buf[11])),
+              fmax3(fmax3(__uint_as_float(buf[12]), __uint_as_float(buf[13]), __uint_as_float(buf[14])),
+                    __uint_as_float(buf[15]), -INFINITY));
+    m *= sl2;
+    float l = 0.f;
+    softmax_step<NB, SEG, 0>(tS, L, sl2, m, l, buf);
+    tmem_wait_st();
+    return l;
+}
+
 } // namespace nle

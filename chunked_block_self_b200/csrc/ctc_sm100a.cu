@@ -68,11 +68,12 @@ __device__ __forceinline__ float chunk_elem(const uint4 &q, int e)
 }
 
 // Per frame: a CTA reads the row's whole 16-byte chunks with 16-byte loads
-// and keeps, per thread, only the largest chunk maximum and the first chunk
-// that reached it (packed bf16 max: about one instruction per logit, so the
-// loop stays under the HBM time); the class inside that chunk is found by
-// reading the chunk once more.  The row's elements before its first 16-byte
-// boundary and after its last one (at most 7 each) are read one by one.
+// and keeps, per thread, only the largest chunk maximum, the first chunk
+// that reached it and that chunk's 8 values (packed bf16 max: about one
+// instruction per logit, so the loop stays under the HBM time); the class
+// inside that chunk is found from the kept values, so no logit is read
+// twice.  The row's elements before its first 16-byte boundary and after its
+// last one (at most 7 each) are read one by one.
 __global__ void __launch_bounds__(kArgmaxThreads)
     ctc_argmax_kernel(const __nv_bfloat16 *__restrict__ logits, long long row_stride, int n_classes,
                       long long total_frames, int32_t *__restrict__ frame_class)
@@ -91,6 +92,7 @@ __global__ void __launch_bounds__(kArgmaxThreads)
 
         float best = -INFINITY;
         int bk = -1;   // first chunk of this thread whose maximum is best (-1: none above -inf)
+        uint4 bq = make_uint4(0u, 0u, 0u, 0u);   // that chunk's values
         int k = tid;
         for (; k + 3 * kArgmaxThreads < nfull; k += 4 * kArgmaxThreads) {
             uint4 q[4];
@@ -103,14 +105,17 @@ __global__ void __launch_bounds__(kArgmaxThreads)
                 if (f > best) {
                     best = f;
                     bk = k + j * kArgmaxThreads;
+                    bq = q[j];
                 }
             }
         }
         for (; k < nfull; k += kArgmaxThreads) {
-            const float f = chunk_max(__ldcs(chunks + k));
+            const uint4 q = __ldcs(chunks + k);
+            const float f = chunk_max(q);
             if (f > best) {
                 best = f;
                 bk = k;
+                bq = q;
             }
         }
 
@@ -118,7 +123,7 @@ __global__ void __launch_bounds__(kArgmaxThreads)
         int bc = INT_MAX;
         if (bk >= 0) {
             // the lowest class of the chunk that holds the maximum
-            const uint4 q = chunks[bk];
+            const uint4 q = bq;
 #pragma unroll
             for (int e = 7; e >= 0; --e)
                 if (chunk_elem(q, e) == best)

@@ -321,6 +321,141 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_kernel(PoolParams
         report(p.status, NLE_ERR_INVALID_ARG);
 }
 
+// ---------------------------------------------------------------- pipelined path
+// For the common shape (windows of at most kPipeMaxP frames, hidden width at
+// most 1024, at most 256 logit classes read as 16-byte chunks) each warp
+// takes a contiguous range of windows and keeps kPipe windows in flight: the
+// frames' hidden rows and logits are copied into a per-warp shared-memory
+// ring with cp.async (16 bytes per lane per copy), so many windows' bytes are
+// on their way from HBM while one is pooled, with no registers held for
+// them.  The arithmetic is the one of posterior_pool_kernel.
+constexpr int kPipe = 3;       // windows in flight per warp
+constexpr int kPipeMaxP = 4;   // frames per window on this path
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolParams p, long long per_warp,
+                                                                          uint32_t slot_bytes)
+{
+    extern __shared__ __align__(16) uint8_t pool_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint8_t *ring = pool_smem + (size_t)warp * (kPipe * slot_bytes + kPipe * sizeof(int2));
+    int2 *hdr = reinterpret_cast<int2 *>(ring + kPipe * slot_bytes);
+    const int n_chunks = p.dim >> 3, z_chunks = p.n_classes >> 3;
+    const uint32_t hid_bytes = (uint32_t)(p.P * p.dim * 2);   // a slot: P hidden rows, then P logit rows
+    const long long gw = (long long)blockIdx.x * kPoolWarps + warp;
+    const long long g0 = gw * per_warp;
+    const long long g1 = g0 + per_warp < p.n_rows ? g0 + per_warp : p.n_rows;
+    if (g0 >= g1)
+        return;
+    PlanWalker w;
+    w.init(p.cu, p.n_seq, p.total, p.P, lane);
+    long long next = g0;   // next window whose copies are issued
+    bool more = true;
+    // copies of window `next` into slot s (or an end mark), as one group
+    auto issue = [&](int s) {
+        int f0 = 0, L = -1, seq;
+        if (more && next < g1 && w.find(next, lane, f0, L, seq)) {
+            uint8_t *slot = ring + (size_t)s * slot_bytes;
+            for (int t = 0; t < L; ++t) {
+                const __nv_bfloat16 *hrow = p.hidden + (long long)(f0 + t) * p.h_stride;
+                for (int ch = lane; ch < n_chunks; ch += 32)
+                    cp_async16(smem_u32(slot + (size_t)(t * p.dim + 8 * ch) * 2), hrow + 8 * ch);
+                if (lane < z_chunks)
+                    cp_async16(smem_u32(slot + hid_bytes + (size_t)(t * p.n_classes + 8 * lane) * 2),
+                               p.logits + (long long)(f0 + t) * p.z_stride + 8 * lane);
+            }
+        } else {
+            more = false;
+            L = -1;
+        }
+        if (lane == 0)
+            hdr[s] = make_int2(f0, L);
+        ++next;
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int s = 0; s < kPipe - 1; ++s)
+        issue(s);
+    for (long long g = g0; g < g1; ++g) {
+        const int s = (int)((g - g0) % kPipe);
+        issue((s + kPipe - 1) % kPipe);   // window g + kPipe - 1, into the slot freed last pass
+        cp_async_wait<kPipe - 1>();       // this lane's copies of window g have landed
+        __syncwarp();
+        const int2 hd = hdr[s];
+        if (hd.y < 0)
+            break;   // past the batch's last window
+        const int f0 = hd.x, L = hd.y;
+        const uint8_t *slot = ring + (size_t)s * slot_bytes;
+        float lw[kPipeMaxP];
+        float M = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < kPipeMaxP; ++t) {
+            lw[t] = -INFINITY;
+            if (t < L) {
+                uint4 q = make_uint4(0u, 0u, 0u, 0u);
+                if (lane < z_chunks)
+                    q = *reinterpret_cast<const uint4 *>(slot + hid_bytes + (size_t)(t * p.n_classes + 8 * lane) * 2);
+                lw[t] = chunk_log_weight(q, p.n_classes, lane);
+                M = fmaxf(M, lw[t]);
+                if (lane == 0 && p.weights)
+                    p.weights[f0 + t] = expf(lw[t]);
+            }
+        }
+        float r[kPipeMaxP];
+        float wsum = 0.f;
+#pragma unroll
+        for (int t = 0; t < kPipeMaxP; ++t) {
+            r[t] = (t < L && M != -INFINITY) ? exp2f((lw[t] - M) * kLog2e) : 0.f;   // 0 for a weight of 0
+            wsum += r[t];
+        }
+        const float inv = M != -INFINITY ? 1.f / wsum : 0.f;   // wsum >= 1 when some weight is not 0
+        __nv_bfloat16 *orow = p.pooled + g * (long long)p.dim;
+        for (int ch = lane; ch < n_chunks; ch += 32) {
+            uint4 res = make_uint4(0u, 0u, 0u, 0u);
+            if (M != -INFINITY) {
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int t = 0; t < kPipeMaxP; ++t) {
+                    if (t < L) {
+                        float v[8];
+                        chunk_vals(*reinterpret_cast<const uint4 *>(slot + (size_t)(t * p.dim + 8 * ch) * 2), v);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            acc[e] = fmaf(r[t], v[e], acc[e]);
+                    }
+                }
+                res = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                                 pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+            }
+            __stcs(reinterpret_cast<uint4 *>(orow + 8 * ch), res);
+        }
+        __syncwarp();   // slot s is refilled by the next pass
+    }
+    cp_async_wait<0>();
+    // the warp holding the last pooled row checks that the batch has no
+    // further window (more windows than rows: nothing past the buffer is
+    // written, the shortfall is reported)
+    if (g1 == p.n_rows) {
+        int a, b, c;
+        if (w.find(p.n_rows, lane, a, b, c) && lane == 0)
+            report(p.status, NLE_ERR_INVALID_ARG);
+    }
+    if (w.bad && lane == 0)
+        report(p.status, NLE_ERR_INVALID_ARG);
+}
+
 } // namespace
 
 extern "C" int nle_posterior_pool_fwd(const void *hidden, int64_t hidden_stride, int dim, const void *logits,
@@ -365,6 +500,24 @@ extern "C" int nle_posterior_pool_fwd(const void *hidden, int64_t hidden_stride,
     // a warp per window; 4 CTAs of 128 threads fit an SM at 128 registers
     const long long ctas = (n_pooled_rows + kPoolWarps - 1) / kPoolWarps, cap = (long long)di.sm_count * 4;
     const int grid = (int)(ctas < cap ? ctas : cap);
+    const bool vec = (reinterpret_cast<uintptr_t>(logits) & 15) == 0 && logits_stride % 8 == 0 && n_classes % 8 == 0;
+    if (vec && n_classes <= 256 && dim <= 1024 && pool_frames <= kPipeMaxP) {
+        const uint32_t slot = (uint32_t)(pool_frames * (dim + n_classes) * 2);
+        const size_t smem_cta = (size_t)kPoolWarps * (kPipe * slot + kPipe * sizeof(int2));
+        int per_sm = (int)((200u * 1024u) / smem_cta);
+        per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+        long long warps = (long long)di.sm_count * per_sm * kPoolWarps;
+        if (warps > n_pooled_rows)
+            warps = n_pooled_rows;
+        const long long per_warp = (n_pooled_rows + warps - 1) / warps;
+        const long long ctas = (warps + kPoolWarps - 1) / kPoolWarps;
+        if (smem_cta > 48 * 1024 && !nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(posterior_pool_pipe_kernel),
+                                                                 dev, di.smem_optin))
+            return NLE_ERR_CUDA;
+        posterior_pool_pipe_kernel<<<(int)ctas, kPoolThreads, smem_cta, static_cast<cudaStream_t>(stream)>>>(
+            p, per_warp, slot);
+        return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
+    }
     // per-warp log weights of a window: above 48 KB (pool_frames > 3072)
     // the kernel needs the opt-in shared memory limit
     const size_t smem = sizeof(float) * kPoolWarps * (size_t)pool_frames;

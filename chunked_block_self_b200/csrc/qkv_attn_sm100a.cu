@@ -1,0 +1,712 @@
+// qkv_attn_sm100a.cu -- the QKV projection fused with varlen block
+// self-attention on B200 (sm_100a).
+//
+// Operation (granite-speech-4.1-2b-nar model card, "Model Architecture" (1)
+// CTC Speech Encoder: each conformer layer's self-attention projects its
+// hidden states to queries, keys and values and attends within 4 s blocks of
+// 200 encoder frames; "Usage / Installation": packed sequences,
+// is_causal=False).  For every block of every packed utterance and every
+// head h:
+//     [Q_h | K_h | V_h] = bf16( X_blk W_h^T + b_h )      (fp32 accumulation)
+//     O_blk,h = softmax(scale * Q_h K_h^T) V_h           (the block kernel)
+// where W_h stacks rows h*64.., H*64 + h*64.. and 2*H*64 + h*64.. (64 each)
+// of the linear layer's weight W [3*H*64][D] (output features x input
+// features), and b the optional bias.  Q, K and V never leave the SM.
+//
+// Design (one persistent CTA per SM, 12 warps; work item = (block, head),
+// dealt round-robin over the CTAs like the block kernel):
+//   warp 0      TMA producer: walks the plan, writes each item's descriptor
+//               into a small ring, and streams the projection operands in
+//               stages of 64 input features: the row tile's X box (128 rows
+//               x 64) and the head's three 64-row W boxes (192 x 64), all
+//               128-byte swizzled, no multicast.  Row tile 0 is block rows
+//               0..127, row tile 1 (blocks longer than 128 frames) rows
+//               128..255.
+//   warp 1      owns TMEM and issues the projection MMAs (lane 0):
+//               D[128 x 192] += X_tile W_h^T, tcgen05.mma kind::f16, M=128,
+//               N=192, K=16 x 4 per stage, fp32 accumulator in TMEM
+//               columns 0..191.
+//   warps 4-7   projection epilogue: per row (TMEM lane) reads D, adds the
+//               bias, rounds to bf16 and writes the row's q, k and v into
+//               shared memory in the layouts the attention MMAs read (Q and
+//               K K-major, V N-major, 128-byte swizzle); rows at or past the
+//               block end are written as zeros.  Then D is released for the
+//               next row tile's projection.
+//   warps 8-11  attention, as one tile warpgroup of the block kernel, on
+//               TMEM columns 256..511: S = Q_x K^T (M=128, N=ceil16(L)),
+//               fp32 register softmax with one shift per row, P (bf16) over
+//               S, O = P V (P from TMEM), O / rowsum rounded to bf16 and
+//               written with warp-contiguous stores through a small staging
+//               buffer; rows past the block end are never written.
+// The projection of the next item runs in its own TMEM columns while the
+// current item's attention runs; the epilogue of the next item's first row
+// tile waits until the current item's last attention MMA has completed
+// (one set of Q/K/V buffers).
+//
+// Every mbarrier wait is bounded (see nle_device.cuh); on expiry the CTA
+// drains its copies and MMAs in flight, frees TMEM and returns.
+#include <cmath>
+
+#include "nle.h"
+#include "attn_softmax.cuh"
+#include "nle_device.cuh"
+#include "nle_host.h"
+
+namespace {
+
+using namespace nle;
+
+constexpr int kThreads = 384;
+constexpr int kEpi0 = 4;           // warps 4-7: projection epilogue
+constexpr int kAttn0 = 8;          // warps 8-11: attention
+constexpr int kSeg = 64;
+constexpr int kQTile = 128;
+constexpr int kRowBytes = 128;     // one frame of one head: 64 bf16
+constexpr uint32_t kXBytes = 128 * 128;          // X box: 128 rows x 64 features
+constexpr uint32_t kWBytes = 192 * 128;          // W boxes: 192 rows x 64 features
+constexpr uint32_t kStageBytes = kXBytes + kWBytes;
+constexpr int kMaxStages = 4;
+constexpr int kDescRing = 8;
+constexpr uint32_t kDescReaders = 9;             // warp 1, epilogue and attention warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kDCol = 0;      // projection accumulator, 192 columns
+constexpr uint32_t kSCol = 256;    // attention: S (<= 256 columns), P over S, O at +128
+constexpr uint32_t kOCol = 128;
+constexpr uint32_t kOutStage = 4 * 2048;         // output staging: 2 KB per attention warp
+
+struct ItemDesc {
+    int f0, L, h, pad;
+};
+
+struct Bars {
+    uint64_t st_full[kMaxStages];
+    uint64_t st_empty[kMaxStages];   // the stage's MMAs have completed
+    uint64_t d_full;                 // the row tile's projection has completed
+    uint64_t d_empty;                // 4 arrivals: the epilogue has read D
+    uint64_t qkv_ready;              // 4 arrivals: the item's Q, K, V are in shared memory
+    uint64_t qkv_free;               // the item's last attention MMA has completed
+    uint64_t desc_full[kDescRing];
+    uint64_t desc_empty[kDescRing];  // every reader has read the entry
+    uint64_t s_full, wg_p, o_full, wg_o;
+    uint64_t mma_done[2];
+    ItemDesc desc[kDescRing];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct Params {
+    const int32_t *cu;
+    int n_seq;
+    int total;
+    int heads;
+    int B;            // block_frames
+    int ksteps;       // input features / 64
+    int nst;          // stage ring depth
+    int qrows;        // rows of the Q buffer (max(NB, 128))
+    uint32_t k_off, v_off, st_off, bars_off, ostage_off;
+    const __nv_bfloat16 *bias;   // nullable, [3 * heads * 64]
+    float scale_log2;
+    __nv_bfloat16 *out;
+    int out_stride;
+    int32_t *status;
+    unsigned long long wait_ns;
+    int flags;
+};
+
+__device__ __forceinline__ uint64_t policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_normal()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// 64 fp32 accumulator columns of this lane's row (+ bias), rounded to bf16
+// and stored as one 128-byte row of a 128-byte-swizzled operand buffer (the
+// 16-byte chunk c of row r sits at chunk position c ^ (r & 7)); zeros when
+// the row lies at or past the block end; nothing stored when `store` is
+// false.  The TMEM loads are warp-collective: every lane of the warp calls
+// this, whatever its row.
+__device__ __forceinline__ void epi_part(uint32_t taddr, const __nv_bfloat16 *bias, bool valid, bool store,
+                                         uint8_t *row_dst, int r)
+{
+    uint32_t v[64];
+    tmem_ld32_nowait(taddr, &v[0]);
+    tmem_ld32_nowait(taddr + 32, &v[32]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+        reg_fence(v[i]);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        float b[8];
+        if (bias) {
+            const uint4 bw = __ldg(reinterpret_cast<const uint4 *>(bias) + c);
+            const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                b[2 * e] = __uint_as_float(bb[e] << 16);
+                b[2 * e + 1] = __uint_as_float(bb[e] & 0xffff0000u);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                b[e] = 0.f;
+        }
+        uint4 q = make_uint4(0, 0, 0, 0);
+        if (valid) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                f[e] = __uint_as_float(v[8 * c + e]) + b[e];
+            q.x = pack_bf16x2(f[0], f[1]);
+            q.y = pack_bf16x2(f[2], f[3]);
+            q.z = pack_bf16x2(f[4], f[5]);
+            q.w = pack_bf16x2(f[6], f[7]);
+        }
+        if (store)
+            *reinterpret_cast<uint4 *>(row_dst + ((c ^ (r & 7)) << 4)) = q;
+    }
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kThreads, 1)
+    qkv_attn_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                    const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t q_base = smem_u32(smem);
+    const uint32_t k_base = q_base + p.k_off;
+    const uint32_t v_base = q_base + p.v_off;
+    const uint32_t st_base = q_base + p.st_off;
+    Bars *bars = reinterpret_cast<Bars *>(smem + p.bars_off);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ------------------------------------------------------------ set-up
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.nst; ++s) {
+            mbar_init(smem_u32(&bars->st_full[s]), 1);
+            mbar_init(smem_u32(&bars->st_empty[s]), 1);
+        }
+        mbar_init(smem_u32(&bars->d_full), 1);
+        mbar_init(smem_u32(&bars->d_empty), 4);
+        mbar_init(smem_u32(&bars->qkv_ready), 4);
+        mbar_init(smem_u32(&bars->qkv_free), 1);
+        for (int j = 0; j < kDescRing; ++j) {
+            mbar_init(smem_u32(&bars->desc_full[j]), 1);
+            mbar_init(smem_u32(&bars->desc_empty[j]), kDescReaders);
+        }
+        mbar_init(smem_u32(&bars->s_full), 1);
+        mbar_init(smem_u32(&bars->wg_p), 4);
+        mbar_init(smem_u32(&bars->o_full), 1);
+        mbar_init(smem_u32(&bars->wg_o), 4);
+        mbar_init(smem_u32(&bars->mma_done[0]), 1);
+        mbar_init(smem_u32(&bars->mma_done[1]), 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 64) {
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_w);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    volatile int *abort_flag = &bars->abort_flag;
+    const unsigned long long wait_ns = p.wait_ns;
+    const int H = p.heads;
+    const int KS = p.ksteps;
+
+    // every reader of the descriptor ring: entry of item n, then release it
+    auto read_desc = [&](int n, ItemDesc &d) -> bool {
+        const int j = n % kDescRing;
+        if (!wait_bar(smem_u32(&bars->desc_full[j]), (uint32_t)(n / kDescRing) & 1, abort_flag, wait_ns, p.status))
+            return false;
+        d = bars->desc[j];
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(smem_u32(&bars->desc_empty[j]));
+        return true;
+    };
+
+    if (warp == 0) {
+        // ==================================================== producer
+        const int step_b = (int)(gridDim.x / H), step_h = (int)(gridDim.x % H);
+        PlanWalker w;
+        w.init(p.cu, p.n_seq, p.total, p.B, lane);
+        const uint64_t pol_x = policy_evict_normal();   // X tiles: read by every head of the block
+        const uint64_t pol_w = policy_evict_last();     // W: read by every item
+        const bool skip0 = (p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) != 0;
+        uint32_t g = 0;   // stages issued
+        int n = 0;        // items published
+        bool ok = true;
+        auto publish = [&](const ItemDesc &d) -> bool {
+            const int j = n % kDescRing;
+            if (n >= kDescRing && !wait_bar(smem_u32(&bars->desc_empty[j]), (uint32_t)(n / kDescRing - 1) & 1,
+                                            abort_flag, wait_ns, p.status))
+                return false;
+            if (lane == 0) {
+                bars->desc[j] = d;
+                mbar_arrive(smem_u32(&bars->desc_full[j]));
+            }
+            __syncwarp();
+            return true;
+        };
+        for (int b = (int)(blockIdx.x / H), h = (int)(blockIdx.x % H);; ++n) {
+            int f0, L, seq;
+            if (!w.find(b, lane, f0, L, seq))
+                break;
+            if (!publish(ItemDesc{f0, L, h, 0})) {
+                ok = false;
+                break;
+            }
+            const int tiles = L > kQTile ? 2 : 1;
+            for (int x = 0; x < tiles && ok; ++x) {
+                for (int kb = 0; kb < KS; ++kb, ++g) {
+                    const int s = (int)(g % (uint32_t)p.nst);
+                    const uint32_t u = g / (uint32_t)p.nst;
+                    if (u > 0 && !wait_bar(smem_u32(&bars->st_empty[s]), (u - 1) & 1, abort_flag, wait_ns, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0 && !(skip0 && g == 0)) {
+                        const uint32_t bar = smem_u32(&bars->st_full[s]);
+                        const uint32_t dst = st_base + (uint32_t)s * kStageBytes;
+                        mbar_arrive_expect_tx(bar, kStageBytes);
+                        tma_load_2d(dst, &tm_x, kb * 64, f0 + x * kQTile, bar, pol_x);
+                        tma_load_2d(dst + kXBytes, &tm_w, kb * 64, h * 64, bar, pol_w);
+                        tma_load_2d(dst + kXBytes + 8192, &tm_w, kb * 64, (H + h) * 64, bar, pol_w);
+                        tma_load_2d(dst + kXBytes + 16384, &tm_w, kb * 64, (2 * H + h) * 64, bar, pol_w);
+                    }
+                    __syncwarp();
+                }
+            }
+            if (!ok)
+                break;
+            b += step_b;
+            h += step_h;
+            if (h >= H) {
+                h -= H;
+                ++b;
+            }
+        }
+        if (w.bad && lane == 0)
+            report(p.status, NLE_ERR_INVALID_ARG);
+        if (ok)
+            publish(ItemDesc{0, -1, 0, 0});   // end marker
+        // drain: the last copies of every stage must land before the CTA exits
+        if (lane == 0) {
+            const uint32_t nst = (uint32_t)p.nst;
+            for (uint32_t m = g > nst ? g - nst : 0; m < g; ++m)
+                if (!(skip0 && m == 0))
+                    wait_bar_drain(smem_u32(&bars->st_full[m % nst]), (m / nst) & 1, wait_ns);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ==================================================== projection MMAs
+        const uint32_t id_p = idesc_bf16_f32(128, 192, false);
+        uint32_t g = 0, tiles_done = 0;
+        for (int n = 0;; ++n) {
+            ItemDesc d;
+            if (!read_desc(n, d) || d.L < 0)
+                break;
+            const int tiles = d.L > kQTile ? 2 : 1;
+            bool ok = true;
+            for (int x = 0; x < tiles && ok; ++x) {
+                if (tiles_done > 0 &&
+                    !wait_bar(smem_u32(&bars->d_empty), (tiles_done - 1) & 1, abort_flag, wait_ns, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < KS; ++kb, ++g) {
+                    const int s = (int)(g % (uint32_t)p.nst);
+                    if (!wait_bar(smem_u32(&bars->st_full[s]), (g / (uint32_t)p.nst) & 1, abort_flag, wait_ns,
+                                  p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a = st_base + (uint32_t)s * kStageBytes;
+                    const uint64_t da = smem_desc_sw128(a, 16, 1024);
+                    const uint64_t db = smem_desc_sw128(a + kXBytes, 16, 1024);
+                    if (lane == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss(tmem + kDCol, da + 2 * kk, db + 2 * kk, id_p, (kb | kk) ? 1u : 0u);
+                        mma_commit(smem_u32(&bars->st_empty[s]));
+                        if (kb == KS - 1)
+                            mma_commit(smem_u32(&bars->d_full));
+                    }
+                    __syncwarp();
+                }
+                ++tiles_done;
+            }
+            if (!ok)
+                break;
+        }
+        if (lane == 0) {
+            mma_commit(smem_u32(&bars->mma_done[0]));
+            wait_bar_drain(smem_u32(&bars->mma_done[0]), 0, wait_ns);
+        }
+        __syncwarp();
+    } else if (warp >= kEpi0 && warp < kAttn0) {
+        // ==================================================== projection epilogue
+        const int qq = warp & 3;
+        const uint32_t tD = tmem + kDCol + ((uint32_t)(qq * 32) << 16);
+        const int NBr = ((p.B + 15) / 16) * 16;   // K and V rows the attention MMAs may read
+        uint32_t tiles_done = 0;
+        for (int n = 0;; ++n) {
+            ItemDesc d;
+            if (!read_desc(n, d) || d.L < 0)
+                break;
+            const int tiles = d.L > kQTile ? 2 : 1;
+            bool ok = true;
+            for (int x = 0; x < tiles; ++x) {
+                if (!wait_bar(smem_u32(&bars->d_full), tiles_done & 1, abort_flag, wait_ns, p.status)) {
+                    ok = false;
+                    break;
+                }
+                // the previous item's attention must be done with Q, K and V
+                if (x == 0 && n > 0 &&
+                    !wait_bar(smem_u32(&bars->qkv_free), (uint32_t)(n - 1) & 1, abort_flag, wait_ns, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int r = x * kQTile + qq * 32 + lane;   // block row of this lane
+                const bool valid = r < d.L;
+                const __nv_bfloat16 *bq = p.bias ? p.bias + (size_t)d.h * 64 : nullptr;
+                const __nv_bfloat16 *bk = p.bias ? p.bias + (size_t)(H + d.h) * 64 : nullptr;
+                const __nv_bfloat16 *bv = p.bias ? p.bias + (size_t)(2 * H + d.h) * 64 : nullptr;
+                // every lane runs the (warp-collective) TMEM loads; only
+                // rows inside the buffers are stored
+                epi_part(tD, bq, valid, r < p.qrows, smem + (size_t)r * kRowBytes, r);
+                epi_part(tD + 64, bk, valid, r < NBr, smem + p.k_off + (size_t)r * kRowBytes, r);
+                epi_part(tD + 128, bv, valid, r < NBr, smem + p.v_off + (size_t)r * kRowBytes, r);
+                fence_proxy_async_smem();   // the rows are read by the async proxy (MMAs)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&bars->d_empty));
+                    if (x == tiles - 1)
+                        mbar_arrive(smem_u32(&bars->qkv_ready));
+                }
+                ++tiles_done;
+            }
+            if (!ok)
+                break;
+        }
+    } else if (warp >= kAttn0) {
+        // ==================================================== attention
+        const int qq = warp & 3;
+        const bool leader = qq == 0;
+        const uint32_t slot = tmem + kSCol;
+        const uint32_t tS = slot + ((uint32_t)(qq * 32) << 16);
+        const float sl2 = p.scale_log2;
+        const uint32_t id_pv = idesc_bf16_f32(128, 64, true);
+        uint8_t *stage = smem + p.ostage_off + (uint32_t)qq * 2048u;
+        int n = -1, x = 1, L = 0, f0 = 0, hcur = 0, nkeys = 16;
+        uint32_t uses = 0;
+        bool ok = true;
+
+        // Next unit: row tile 1 of the item if it has one, else row tile 0
+        // of the next item; the leader issues the unit's S MMA once the
+        // previous unit's O has been read and, for a new item, its Q, K and
+        // V are in shared memory.
+        auto advance = [&]() -> bool {
+            if (!(x == 0 && L > kQTile)) {
+                ++n;
+                ItemDesc d;
+                if (!read_desc(n, d)) {
+                    ok = false;
+                    return false;
+                }
+                if (d.L < 0)
+                    return false;
+                f0 = d.f0;
+                L = d.L;
+                hcur = d.h;
+                x = 0;
+                nkeys = (L + 15) & ~15;
+            } else {
+                x = 1;
+            }
+            if (leader) {
+                if (uses > 0 && !wait_bar(smem_u32(&bars->wg_o), (uses - 1) & 1, abort_flag, wait_ns, p.status)) {
+                    ok = false;
+                    return false;
+                }
+                if (x == 0 && !wait_bar(smem_u32(&bars->qkv_ready), (uint32_t)n & 1, abort_flag, wait_ns, p.status)) {
+                    ok = false;
+                    return false;
+                }
+                tc_fence_after();
+                const uint64_t da = smem_desc_sw128(q_base + (uint32_t)(x * kQTile * kRowBytes), 16, 1024);
+                const uint64_t db = smem_desc_sw128(k_base, 16, 1024);
+                const uint32_t id_s = idesc_bf16_f32(128, nkeys, false);
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(slot, da + 2 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
+                    mma_commit(smem_u32(&bars->s_full));
+                }
+                __syncwarp();
+            }
+            return true;
+        };
+
+        uint32_t pk[32];
+        bool pending = false;
+        int ef0 = 0, eL = 0, eh = 0, erow0 = 0;
+        for (;;) {
+            const bool have = advance();
+            if (!ok)
+                break;
+            if (pending) {
+                // 16 rows at a time through the staging buffer, then four
+                // whole 128-byte rows per store instruction; rows past the
+                // block end are never written
+                const int rows_left = eL - erow0;
+                __nv_bfloat16 *obase = p.out + (size_t)(ef0 + erow0) * p.out_stride + eh * 64;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    if (half * 16 < rows_left) {
+                        if ((lane >> 4) == half) {
+                            const int r = lane & 15;
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                *reinterpret_cast<uint4 *>(stage + r * 128 + ((c ^ (r & 7)) << 4)) =
+                                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int r = 4 * i + (lane >> 3), c = lane & 7;
+                            if (half * 16 + r < rows_left) {
+                                const uint4 val =
+                                    *reinterpret_cast<const uint4 *>(stage + r * 128 + ((c ^ (r & 7)) << 4));
+                                *reinterpret_cast<uint4 *>(obase + (size_t)(half * 16 + r) * p.out_stride + c * 8) =
+                                    val;
+                            }
+                        }
+                        __syncwarp();
+                    }
+                }
+                pending = false;
+            }
+            if (!have)
+                break;
+            // ---------------------------------------------- softmax
+            if (!wait_bar(smem_u32(&bars->s_full), uses & 1, abort_flag, wait_ns, p.status))
+                break;
+            tc_fence_after();
+            const int row0 = x * kQTile + qq * 32;
+            const bool active = row0 < L;
+            float l = 1.f;
+            if (active)
+                l = block_softmax_rows<NB, kSeg>(tS, L, sl2);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bars->wg_p));
+            // ---------------------------------------------- O = P V
+            if (leader) {
+                if (!wait_bar(smem_u32(&bars->wg_p), uses & 1, abort_flag, wait_ns, p.status))
+                    break;
+                tc_fence_after();
+                // V rows L..nkeys-1 are zeros (written so by the epilogue)
+                const uint64_t dv = smem_desc_sw128(v_base, 0, 1024);
+                if (lane == 0) {
+                    const int ksteps = nkeys / 16;
+#pragma unroll
+                    for (int kk = 0; kk < NB / 16; ++kk)
+                        if (kk < ksteps)
+                            mma_ts(slot + kOCol, slot + kk * 8, dv + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
+                                   kk > 0 ? 1u : 0u);
+                    mma_commit(smem_u32(&bars->o_full));
+                    if (x == 1 || L <= kQTile)   // the item's last MMA: Q, K and V may be overwritten
+                        mma_commit(smem_u32(&bars->qkv_free));
+                }
+                __syncwarp();
+            }
+            // ---------------------------------------------- read O
+            if (!wait_bar(smem_u32(&bars->o_full), uses & 1, abort_flag, wait_ns, p.status))
+                break;
+            tc_fence_after();
+            if (active) {
+                uint32_t o[64];
+                tmem_ld32_nowait(tS + kOCol, &o[0]);
+                tmem_ld32_nowait(tS + kOCol + 32, &o[32]);
+                tmem_wait_ld();
+                const float inv = 1.f / l;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    reg_fence(o[2 * i]);
+                    reg_fence(o[2 * i + 1]);
+                    pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bars->wg_o));
+            ++uses;
+            pending = active;
+            ef0 = f0;
+            eL = L;
+            eh = hcur;
+            erow0 = row0;
+        }
+        if (leader) {
+            if (lane == 0) {
+                mma_commit(smem_u32(&bars->mma_done[1]));
+                wait_bar_drain(smem_u32(&bars->mma_done[1]), 0, wait_ns);
+            }
+            __syncwarp();
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+using QkvKernel = void (*)(CUtensorMap, CUtensorMap, Params);
+
+template <int NB>
+QkvKernel qkv_kernel_nb()
+{
+    return reinterpret_cast<QkvKernel>(qkv_attn_kernel<NB>);
+}
+
+QkvKernel pick_qkv_kernel(int nb)
+{
+    switch (nb) {
+    case 16: return qkv_kernel_nb<16>();
+    case 32: return qkv_kernel_nb<32>();
+    case 48: return qkv_kernel_nb<48>();
+    case 64: return qkv_kernel_nb<64>();
+    case 80: return qkv_kernel_nb<80>();
+    case 96: return qkv_kernel_nb<96>();
+    case 112: return qkv_kernel_nb<112>();
+    case 128: return qkv_kernel_nb<128>();
+    case 144: return qkv_kernel_nb<144>();
+    case 160: return qkv_kernel_nb<160>();
+    case 176: return qkv_kernel_nb<176>();
+    case 192: return qkv_kernel_nb<192>();
+    case 208: return qkv_kernel_nb<208>();
+    case 224: return qkv_kernel_nb<224>();
+    case 240: return qkv_kernel_nb<240>();
+    default: return qkv_kernel_nb<256>();
+    }
+}
+
+} // namespace
+
+extern "C" int nle_block_attn_qkv_fwd_ex(const void *x, const void *w_qkv, const void *bias, void *out,
+                                         const int32_t *cu_seqlens, int n_seq, int64_t total_frames, int d_model,
+                                         int heads, int d_head, int block_frames, float softmax_scale,
+                                         int32_t *dev_status, int flags, int64_t wait_limit_ns, void *stream)
+{
+    if (n_seq < 0 || total_frames < 0 || heads <= 0 || block_frames <= 0 || d_model <= 0 || wait_limit_ns < 0)
+        return NLE_ERR_INVALID_ARG;
+    if (d_head != 64 || block_frames > 256 || d_model % 64 != 0 || d_model > 16384 ||
+        total_frames > 0x7fffffffLL || (int64_t)3 * heads * 64 > 0x7fffffffLL)
+        return NLE_ERR_UNSUPPORTED;
+    const long long max_items = ((long long)n_seq + total_frames / block_frames) * heads;
+    if (max_items > 0x7fffffffLL)
+        return NLE_ERR_UNSUPPORTED;
+    if (n_seq == 0 || total_frames == 0)
+        return NLE_OK;
+    if (!x || !w_qkv || !out || !cu_seqlens)
+        return NLE_ERR_INVALID_ARG;
+    if (!nle::aligned16(x) || !nle::aligned16(w_qkv) || !nle::aligned16(out) || (bias && !nle::aligned16(bias)))
+        return NLE_ERR_MISALIGNED;
+
+    nle::DeviceInfo di;
+    int dev = 0;
+    if (!nle::current_device_info(&di, &dev))
+        return NLE_ERR_CUDA;
+    if (di.cc_major != 10)
+        return NLE_ERR_UNSUPPORTED;
+
+    const int B = block_frames;
+    const int NB = (B + 15) / 16 * 16;
+    Params p{};
+    p.cu = cu_seqlens;
+    p.n_seq = n_seq;
+    p.total = (int)total_frames;
+    p.heads = heads;
+    p.B = B;
+    p.ksteps = d_model / 64;
+    // Q holds >= 128 rows (each S MMA reads 128 rows from its tile's base;
+    // row tile 1 reads past the Q rows into the K buffer, rows it ignores)
+    p.qrows = NB > kQTile ? NB : kQTile;
+    const uint32_t q_bytes = (uint32_t)p.qrows * kRowBytes, kv_bytes = (uint32_t)NB * kRowBytes;
+    p.k_off = q_bytes;
+    p.v_off = q_bytes + kv_bytes;
+    p.st_off = (q_bytes + 2 * kv_bytes + 1023) & ~1023u;
+    const size_t bars_round = ((sizeof(Bars) + 127) / 128) * 128;
+    int nst = 0;
+    for (int s = kMaxStages; s >= 2; --s)
+        if ((size_t)p.st_off + (size_t)s * kStageBytes + bars_round + kOutStage + 1024 <= (size_t)di.smem_optin) {
+            nst = s;
+            break;
+        }
+    if (!nst)
+        return NLE_ERR_UNSUPPORTED;
+    p.nst = nst;
+    p.bars_off = p.st_off + (uint32_t)nst * kStageBytes;
+    p.ostage_off = p.bars_off + (uint32_t)bars_round;
+    size_t smem = (size_t)p.ostage_off + kOutStage + 1024;
+    // one CTA per SM: it owns all 512 TMEM columns
+    if (smem <= (size_t)di.smem_optin / 2)
+        smem = (size_t)di.smem_optin / 2 + 1024;
+    p.bias = static_cast<const __nv_bfloat16 *>(bias);
+    const double scale = softmax_scale > 0.f ? (double)softmax_scale : 1.0 / std::sqrt((double)d_head);
+    p.scale_log2 = (float)(scale * 1.4426950408889634);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.out_stride = heads * 64;
+    p.status = dev_status;
+    p.wait_ns = wait_limit_ns > 0 ? (unsigned long long)wait_limit_ns : 1000000000ull;
+    p.flags = flags;
+
+    CUtensorMap tx, tw;
+    if (!nle::encode_tmap_bf16_2d(&tx, x, (uint64_t)d_model, (uint64_t)total_frames, (uint64_t)d_model, 64, 128) ||
+        !nle::encode_tmap_bf16_2d(&tw, w_qkv, (uint64_t)d_model, (uint64_t)3 * heads * 64, (uint64_t)d_model, 64,
+                                  64))
+        return NLE_ERR_CUDA;
+
+    const QkvKernel kern = pick_qkv_kernel(NB);
+    if (!nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(kern), dev, di.smem_optin))
+        return NLE_ERR_CUDA;
+    const int grid = (int)(max_items < di.sm_count ? max_items : di.sm_count);
+    kern<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tx, tw, p);
+    return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
+}
+
+extern "C" int nle_block_attn_qkv_fwd(const void *x, const void *w_qkv, const void *bias, void *out,
+                                      const int32_t *cu_seqlens, int n_seq, int64_t total_frames, int d_model,
+                                      int heads, int d_head, int block_frames, void *stream)
+{
+    return nle_block_attn_qkv_fwd_ex(x, w_qkv, bias, out, cu_seqlens, n_seq, total_frames, d_model, heads, d_head,
+                                     block_frames, 0.f, nullptr, 0, 0, stream);
+}

@@ -50,6 +50,9 @@ _SIGS = {
     "nle_block_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int, _vp], _int),
     "nle_block_attn_fwd_ex": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int, _f32, _i64, _vp,
                                _int, _i64, _vp], _int),
+    "nle_block_attn_qkv_fwd": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int, _int, _vp], _int),
+    "nle_block_attn_qkv_fwd_ex": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _int, _int, _f32, _vp, _int,
+                                   _i64, _vp], _int),
     "nle_window_xattn_fwd": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _int, _int, _int, _int, _vp], _int),
     "nle_window_xattn_fwd_ex": ([_vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _int, _int, _int, _int, _f32,
                                  _vp, _int, _i64, _vp], _int),
@@ -164,6 +167,57 @@ def block_attn(q, k, v, cu_seqlens, block_frames: int = 200, out=None, stream=No
     if out is None:
         out = torch.empty_like(q)
     nle_block_attn_fwd(q, k, v, out, cu_seqlens, block_frames=block_frames, stream=stream)
+    return out
+
+
+# ------------------------------------------------------------------ QKV projection + block attention
+def nle_block_attn_qkv_fwd_ex(x, w_qkv, bias, out, cu_seqlens, n_seq: int | None = None,
+                              total_frames: int | None = None, heads: int | None = None, d_head: int = 64,
+                              block_frames: int = 200, softmax_scale: float = 0.0, dev_status=None, flags: int = 0,
+                              wait_limit_ns: int = 0, stream=None) -> None:
+    """x: CUDA bf16 [frames, d_model]; w_qkv: bf16 [3 * heads * 64, d_model];
+    bias: None or bf16 [3 * heads * 64]; out: bf16 [frames, heads, 64]."""
+    _dev_tensor(x, "x", torch.bfloat16)
+    _dev_tensor(w_qkv, "w_qkv", torch.bfloat16)
+    _dev_tensor(out, "out", torch.bfloat16)
+    if bias is not None:
+        _dev_tensor(bias, "bias", torch.bfloat16)
+    _dev_tensor(cu_seqlens, "cu_seqlens", torch.int32)
+    if dev_status is not None:
+        _dev_tensor(dev_status, "dev_status", torch.int32)
+    if x.dim() != 2 or not x.is_contiguous() or not w_qkv.is_contiguous():
+        raise ValueError("x: contiguous [frames, d_model]; w_qkv: contiguous [3 * heads * 64, d_model]")
+    n_seq = cu_seqlens.numel() - 1 if n_seq is None else n_seq
+    total_frames = x.shape[0] if total_frames is None else total_frames
+    heads = out.shape[1] if heads is None else heads
+    _check(_lib.nle_block_attn_qkv_fwd_ex(_ptr(x), _ptr(w_qkv), _ptr(bias), _ptr(out), _ptr(cu_seqlens), n_seq,
+                                          total_frames, x.shape[1], heads, d_head, block_frames,
+                                          float(softmax_scale), _ptr(dev_status), flags, wait_limit_ns,
+                                          _stream(stream)),
+           "nle_block_attn_qkv_fwd_ex")
+
+
+def nle_block_attn_qkv_fwd(x, w_qkv, bias, out, cu_seqlens, block_frames: int = 200, stream=None) -> None:
+    _dev_tensor(x, "x", torch.bfloat16)
+    _dev_tensor(w_qkv, "w_qkv", torch.bfloat16)
+    _dev_tensor(out, "out", torch.bfloat16)
+    if bias is not None:
+        _dev_tensor(bias, "bias", torch.bfloat16)
+    _dev_tensor(cu_seqlens, "cu_seqlens", torch.int32)
+    if x.dim() != 2 or not x.is_contiguous() or not w_qkv.is_contiguous():
+        raise ValueError("x: contiguous [frames, d_model]; w_qkv: contiguous [3 * heads * 64, d_model]")
+    _check(_lib.nle_block_attn_qkv_fwd(_ptr(x), _ptr(w_qkv), _ptr(bias), _ptr(out), _ptr(cu_seqlens),
+                                       cu_seqlens.numel() - 1, x.shape[0], x.shape[1], out.shape[1], 64,
+                                       block_frames, _stream(stream)),
+           "nle_block_attn_qkv_fwd")
+
+
+def block_attn_qkv(x, w_qkv, cu_seqlens, heads: int, bias=None, block_frames: int = 200, out=None,
+                   stream=None) -> torch.Tensor:
+    """O [frames, heads, 64] of block attention of X's QKV projection."""
+    if out is None:
+        out = torch.empty((x.shape[0], heads, 64), dtype=torch.bfloat16, device=x.device)
+    nle_block_attn_qkv_fwd(x, w_qkv, bias, out, cu_seqlens, block_frames=block_frames, stream=stream)
     return out
 
 

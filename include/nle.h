@@ -127,6 +127,46 @@ int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v,
                           int flags, int64_t wait_limit_ns, void *stream);
 
 /* ---------------------------------------------------------------------
+ * QKV projection fused with block self-attention (model card, "Model
+ * Architecture" (1): each encoder layer's self-attention projects its
+ * hidden states to queries, keys and values and attends within 4 s blocks).
+ * For every block and head h:
+ *     [Q_h | K_h | V_h] = bf16(X_blk W_h^T + b_h)  (fp32 accumulation, one
+ *                                                   rounding to bf16)
+ *     O_blk,h = softmax(scale * Q_h K_h^T) V_h     (as nle_block_attn_fwd)
+ * Q, K and V are formed on chip and never written to memory.
+ *
+ * x              device bf16 [total_frames][d_model], dense rows
+ * w_qkv          device bf16 [3 * heads * 64][d_model]: a linear layer's
+ *                weight (output features x input features); rows
+ *                [0, H*64) give Q, [H*64, 2*H*64) K, [2*H*64, 3*H*64) V,
+ *                head h taking rows h*64 .. h*64+63 of each
+ * bias           nullable device bf16 [3 * heads * 64], same row order
+ * out            device bf16 [total_frames][heads][64]
+ * cu_seqlens     device int32 [n_seq + 1] (as nle_block_attn_fwd)
+ * d_model        input features: a multiple of 64, at most 16384
+ * heads, d_head  heads >= 1, d_head must be 64
+ * block_frames   1..256 (200 for 4 s at 50 Hz)
+ * x, w_qkv, bias and out must be 16-byte aligned.  Errors as
+ * nle_block_attn_fwd (NLE_ERR_UNSUPPORTED also for d_model not a multiple
+ * of 64 or above 16384).  No allocation; asynchronous on `stream`.
+ * The _ex form adds softmax_scale (<= 0: 1/sqrt(d_head)), dev_status, flags
+ * and wait_limit_ns, as nle_block_attn_fwd_ex.
+ */
+int nle_block_attn_qkv_fwd(const void *x, const void *w_qkv, const void *bias,
+                           void *out, const int32_t *cu_seqlens, int n_seq,
+                           int64_t total_frames, int d_model, int heads,
+                           int d_head, int block_frames, void *stream);
+
+int nle_block_attn_qkv_fwd_ex(const void *x, const void *w_qkv,
+                              const void *bias, void *out,
+                              const int32_t *cu_seqlens, int n_seq,
+                              int64_t total_frames, int d_model, int heads,
+                              int d_head, int block_frames,
+                              float softmax_scale, int32_t *dev_status,
+                              int flags, int64_t wait_limit_ns, void *stream);
+
+/* ---------------------------------------------------------------------
  * Windowed cross-attention (model card, "Model Architecture" (2)).
  *
  * q, out          device bf16 [n_query_rows][heads][64]; n_query_rows must be

@@ -87,3 +87,26 @@ def test_binding_rejects_cpu_tensors():
     cu = torch.tensor([0, 4], dtype=torch.int32)
     with pytest.raises(TypeError):
         nle.nle_block_attn_fwd(x, x, x, x, cu)
+
+
+def _qkv(**kw):
+    a = dict(x=16, w=16, b=None, out=16, cu=16, n_seq=1, total=400, dm=1024, heads=16, d=64, B=200)
+    a.update(kw)
+    return nle._lib.nle_block_attn_qkv_fwd(a["x"], a["w"], a["b"], a["out"], a["cu"], a["n_seq"], a["total"],
+                                           a["dm"], a["heads"], a["d"], a["B"], None)
+
+
+def test_block_attn_qkv_host_validation():
+    assert _qkv(d=32) == nle.NLE_ERR_UNSUPPORTED
+    assert _qkv(dm=1000) == nle.NLE_ERR_UNSUPPORTED        # not a multiple of 64
+    assert _qkv(dm=16384 + 64) == nle.NLE_ERR_UNSUPPORTED
+    assert _qkv(dm=0) == nle.NLE_ERR_INVALID_ARG
+    assert _qkv(B=257) == nle.NLE_ERR_UNSUPPORTED
+    assert _qkv(B=0) == nle.NLE_ERR_INVALID_ARG
+    assert _qkv(heads=0) == nle.NLE_ERR_INVALID_ARG
+    assert _qkv(x=None) == nle.NLE_ERR_INVALID_ARG
+    assert _qkv(w=None) == nle.NLE_ERR_INVALID_ARG
+    assert _qkv(x=24) == nle.NLE_ERR_MISALIGNED
+    assert _qkv(b=8) == nle.NLE_ERR_MISALIGNED              # bias, when given, 16-byte aligned too
+    assert _qkv(n_seq=0, x=None, w=None, out=None, cu=None) == nle.NLE_OK
+    assert _qkv(total=0) == nle.NLE_OK

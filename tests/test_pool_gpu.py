@@ -78,7 +78,10 @@ def test_golden_cases(case, cuda_device):
 
 @pytest.mark.parametrize("P,dim,n_classes,pads", [
     (2, 1024, 256, (0, 0)), (1, 8, 1, (0, 0)), (2, 8, 2, (8, 1)), (3, 24, 37, (16, 3)), (4, 1024, 256, (8, 5)),
-    (7, 64, 1000, (0, 7)), (2, 1032, 2, (0, 0)), (16, 128, 5, (0, 2))])
+    (7, 64, 1000, (0, 7)), (2, 1032, 2, (0, 0)), (16, 128, 5, (0, 2)),
+    # the pipelined path (P <= 4, dim <= 1024, classes <= 256 in 16-byte chunks)
+    (1, 1024, 256, (0, 0)), (3, 64, 8, (8, 8)), (4, 1024, 256, (8, 0)), (2, 8, 16, (0, 0)),
+    (4, 1000, 248, (16, 8))])
 def test_random_shapes(P, dim, n_classes, pads, cuda_device):
     lengths = [37, 0, 1, 200, 5, 64, 3]
     cu = wl.cu_seqlens(lengths)
@@ -87,13 +90,14 @@ def test_random_shapes(P, dim, n_classes, pads, cuda_device):
     _check(x, cu, cuda_device, P, dim, n_classes)
 
 
-def test_degenerate_weights(cuda_device):
+@pytest.mark.parametrize("C", [6, 8])   # the general and the pipelined path
+def test_degenerate_weights(C, cuda_device):
     """Only the blank (every weight 0 -> zero rows), a -inf blank (weight
     exactly 1), and a blank far above the rest (weights below fp32's range;
     their window is still their weighted mean)."""
     lengths = [6, 4, 5]
     cu = wl.cu_seqlens(lengths)
-    T, C, D = 15, 6, 16
+    T, D = 15, 16
     rng = np.random.default_rng(7)
     z = rng.standard_normal((T, C)).astype(np.float32)
     z[0:6, 1:] = -np.inf          # utterance 0: every weight 0
@@ -108,13 +112,14 @@ def test_degenerate_weights(cuda_device):
     assert np.all(gw[6:8] == 1.0)
 
 
-def test_rows_short_reported_and_untouched(cuda_device):
+@pytest.mark.parametrize("n_classes", [4, 8])   # the general and the pipelined path
+def test_rows_short_reported_and_untouched(n_classes, cuda_device):
     """Too few pooled rows for the windows: rows past the buffer are never
     written and the status says so."""
     nle = _nle()
     lengths = [9, 7]
     cu = wl.cu_seqlens(lengths)
-    x = wl.pool_inputs(lengths, 16, 4, seed=5)
+    x = wl.pool_inputs(lengths, 16, n_classes, seed=5)
     n_rows = int(oracle.pooled_rows(cu, 2)[-1])
     guard = torch.full((n_rows + 4, 16), 7.0, dtype=torch.bfloat16, device=cuda_device)
     status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
@@ -129,9 +134,10 @@ def test_rows_short_reported_and_untouched(cuda_device):
     _compare(short.float().cpu().double().numpy(), ref[:n_rows - 3])
 
 
-def test_invalid_offsets_reported(cuda_device):
+@pytest.mark.parametrize("n_classes", [4, 8])   # the general and the pipelined path
+def test_invalid_offsets_reported(n_classes, cuda_device):
     nle = _nle()
-    x = wl.pool_inputs([8], 16, 4, seed=6)
+    x = wl.pool_inputs([8], 16, n_classes, seed=6)
     cu_bad = torch.tensor([0, 9], dtype=torch.int32, device=cuda_device)   # past total_frames
     out = torch.full((4, 16), 7.0, dtype=torch.bfloat16, device=cuda_device)
     status = torch.zeros(1, dtype=torch.int32, device=cuda_device)

@@ -7,20 +7,12 @@
 // for every block of every packed utterance and every head,
 //     O = softmax(scale * Q K^T) V  over the block's L <= B frames.
 //
-// Items are dealt round-robin over the CTAs, every whole block of the batch
-// first and the utterances' partial last blocks after them, so each CTA
-// meets large items first and ends on small ones.
-//
 // Design (one persistent CTA per SM, three warpgroups):
 //   warps 0, 1  TMA producers.  Work item = (block, head).  Warp 0 loads
 //               Q (two boxes: rows 0..127 and 128..B-1) and K of each item
 //               into a ring of QK stages, warp 1 loads V into a ring of V
 //               stages, all as 128-byte-swizzled TMA boxes (no multicast).
-//               Warp 0 is the only role of the Q/K side that walks the plan:
-//               it writes each item's descriptor (first frame, length, head)
-//               into a small ring next to the item's loads, and end markers
-//               after the last item.  Warp 1 also owns TMEM (allocates and
-//               frees it).
+//               Warp 1 also owns TMEM (allocates and frees it).
 //   warps 4-7   tile warpgroup 0, TMEM slot 0: the CTA's even items,
 //   warps 8-11  tile warpgroup 1, TMEM slot 1: the odd items.  For each of
 //               its items a warpgroup computes row tile 0 (block rows
@@ -42,12 +34,10 @@
 //               64-column register segments: p = exp2(S*scale*log2e
 //               - m) in fp32 with one shift m per row (keys >= L are 0 by
 //               index, never by value), row sum, bf16 pack, P written back
-//               over S.  The epilogue reads O (then releases the slot for
-//               the next S MMA), divides by the row sum, rounds to bf16 and
-//               writes each row < L through a small shared-memory staging
-//               buffer with warp-contiguous 16-byte stores (four whole rows
-//               per store instruction), while the warpgroup's next S MMA
-//               runs.  Rows past the block end are never written.
+//               over S.  The epilogue reads O, divides by the row sum,
+//               rounds to bf16 and writes each row < L with 16-byte vector
+//               stores, while the warpgroup's next S MMA runs.  Rows past the
+//               block end are never written.
 //               QK and V rings have even depths, so an item's stages have
 //               the parity of its warpgroup and each stage belongs to one
 //               warpgroup.
@@ -103,15 +93,6 @@ constexpr int kMaxV = 4;           // V ring depth upper bound
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256; // TMEM columns per tile slot
 constexpr uint32_t kOCol = 128;     // O offset inside a tile slot
-constexpr uint32_t kStageBytes = 8 * 2048;   // output staging: 2 KB per tile warp
-
-// Item descriptor, written by the Q/K producer next to the item's loads
-// (ring of kDescRing entries, item n in entry n % kDescRing): first frame,
-// length (-1: no more items for the reader) and head.
-struct ItemDesc {
-    int f0, L, h, pad;
-};
-constexpr int kDescRing = 2 * kMaxQK;
 
 struct Bars {
     uint64_t qk_full[kMaxQK];
@@ -123,8 +104,6 @@ struct Bars {
     uint64_t o_full[2];
     uint64_t wg_o[2];            // 4 arrivals: O of the unit read from TMEM
     uint64_t mma_done[2];
-    uint64_t desc_ready[2];      // the leader has read the slot's next item descriptor
-    ItemDesc desc[kDescRing];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -143,7 +122,6 @@ struct Params {
     uint32_t qk_bytes;  // QK stage
     uint32_t v_bytes;   // V stage
     uint32_t bars_off;  // barriers, after the QK and V rings
-    uint32_t stage_off; // output staging (2 KB per tile warp), after the barriers
     float scale_log2;
     __nv_bfloat16 *out;
     int out_stride;     // elements between output frames (heads * 64)
@@ -182,7 +160,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&bars->o_full[t]), 1);
             mbar_init(smem_u32(&bars->wg_o[t]), 4);
             mbar_init(smem_u32(&bars->mma_done[t]), 1);
-            mbar_init(smem_u32(&bars->desc_ready[t]), 1);
         }
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -221,19 +198,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ==================================================== producers
         // Warp 0 loads Q and K of every item, warp 1 loads V; each refills a
         // stage as soon as the stage's last reader has released it (QK: the
-        // item's last S MMA; V: its last PV MMA).  Warp 0 also writes each
-        // item's descriptor (first frame, length, head) into the descriptor
-        // ring before arming the item's stage, so the tile warpgroups never
-        // walk the plan themselves; after the last item it publishes two
-        // end markers (one for each warpgroup's next item).
+        // item's last S MMA; V: its last PV MMA).
         const bool is_v = warp == 1;
         const int nst = is_v ? p.nsv : p.sqk;
-        WholeFirstWalker w;
+        PlanWalker w;
         w.init(p.cu, p.n_seq, p.total, p.B, lane);
         const uint64_t pol = policy_evict_first();
         const bool skip0 = !is_v && (p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) != 0;
         int n = 0;   // items whose copies were issued
-        bool ok = true;
         for (int b = first_b, h = first_h;; ++n) {
             int f0, L, seq;
             if (!w.find(b, lane, f0, L, seq))
@@ -241,28 +213,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = n % nst;
             const uint32_t u = (uint32_t)(n / nst);
             if (u > 0 && !wait_bar(smem_u32(is_v ? &bars->v_empty[s] : &bars->qk_empty[s]), (u - 1) & 1, abort_flag,
-                                   wait_ns, p.status)) {
-                ok = false;
+                                   wait_ns, p.status))
                 break;
-            }
             if (lane == 0) {
                 if (is_v) {
                     const uint32_t bar = smem_u32(&bars->v_full[s]);
                     mbar_arrive_expect_tx(bar, p.B * kRowBytes);
                     tma_load_2d(v_base + s * p.v_bytes, &tm_v, h * 64, f0, bar, pol);
-                } else {
-                    bars->desc[n % kDescRing] = ItemDesc{f0, L, h, 0};
-                    if (!(skip0 && n == 0)) {
-                        const bool two = L > kQTile;
-                        const uint32_t bar = smem_u32(&bars->qk_full[s]);
-                        const uint32_t bytes = (p.q0rows + (two ? p.q1rows : 0) + p.B) * kRowBytes;
-                        const uint32_t qdst = qk_base + s * p.qk_bytes;
-                        mbar_arrive_expect_tx(bar, bytes);
-                        tma_load_2d(qdst, &tm_q0, h * 64, f0, bar, pol);
-                        if (two)
-                            tma_load_2d(qdst + kQTile * kRowBytes, &tm_q1, h * 64, f0 + kQTile, bar, pol);
-                        tma_load_2d(qdst + p.q_bytes, &tm_k, h * 64, f0, bar, pol);
-                    }
+                } else if (!(skip0 && n == 0)) {
+                    const bool two = L > kQTile;
+                    const uint32_t bar = smem_u32(&bars->qk_full[s]);
+                    const uint32_t bytes = (p.q0rows + (two ? p.q1rows : 0) + p.B) * kRowBytes;
+                    const uint32_t qdst = qk_base + s * p.qk_bytes;
+                    mbar_arrive_expect_tx(bar, bytes);
+                    tma_load_2d(qdst, &tm_q0, h * 64, f0, bar, pol);
+                    if (two)
+                        tma_load_2d(qdst + kQTile * kRowBytes, &tm_q1, h * 64, f0 + kQTile, bar, pol);
+                    tma_load_2d(qdst + p.q_bytes, &tm_k, h * 64, f0, bar, pol);
                 }
                 NLE_TRACE_AT(0, n, is_v ? 1 : 0);
             }
@@ -276,29 +243,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!is_v && w.bad && lane == 0)
             report(p.status, NLE_ERR_INVALID_ARG);
-        // end markers for items n and n + 1 (each warpgroup learns that it
-        // has no further item); each waits for its stage like a real item,
-        // which also proves that the stage's previous copies have landed
-        int sent = 0;
-        if (!is_v && ok) {
-            for (; sent < 2; ++sent) {
-                const int m = n + sent, s = m % nst;
-                const uint32_t u = (uint32_t)(m / nst);
-                if (u > 0 && !wait_bar(smem_u32(&bars->qk_empty[s]), (u - 1) & 1, abort_flag, wait_ns, p.status))
-                    break;
-                if (lane == 0) {
-                    bars->desc[m % kDescRing] = ItemDesc{0, -1, 0, 0};
-                    mbar_arrive(smem_u32(&bars->qk_full[s]));
-                }
-                __syncwarp();
-            }
-        }
         // drain: every issued copy must land before the CTA can exit.
         // Copies went to stages round-robin, so the last ones to each stage
-        // are those of the final min(n, stages) items; the stages that took
-        // an end marker are known to be complete.
+        // are those of the final min(n, stages) items.
         if (lane == 0) {
-            for (int m = n - nst + sent; m < n; ++m)
+            for (int m = n - nst; m < n; ++m)
                 if (m >= 0 && !(skip0 && m == 0))
                     wait_bar_drain(smem_u32(is_v ? &bars->v_full[m % nst] : &bars->qk_full[m % nst]),
                                    (uint32_t)(m / nst) & 1, wait_ns);
@@ -315,9 +264,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // warpgroups thus run independent chains, and one's MMA and output
         // phases overlap the other's softmax.  The first warp's elected lane
         // issues the slot's MMAs; all four warps run softmax and epilogue.
-        // Items come from the descriptor ring: the leader reads item n's
-        // entry once its QK stage is full and tells the other three warps
-        // through desc_ready.
         const int t = (warp - kSoftmax0) >> 2;     // TMEM slot
         const int qq = warp & 3;                   // TMEM lane quarter of this warp
         const bool leader = qq == 0;
@@ -325,13 +271,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tS = slot + ((uint32_t)(qq * 32) << 16);
         const float sl2 = p.scale_log2;
         const uint32_t id_pv = idesc_bf16_f32(128, 64, true);
-        // 2 KB of output staging for this warp: 16 rows of 128 B, the
-        // 16-byte chunks of row r at chunk positions c ^ (r & 7)
-        uint8_t *stage = smem + p.stage_off + (uint32_t)(warp - kSoftmax0) * 2048u;
-        int n = t - 2;       // current item
+        PlanWalker w;
+        w.init(p.cu, p.n_seq, p.total, p.B, lane);
+        // the CTA's item sequence: item n is blockIdx.x + n * gridDim.x
+        int b = first_b, h = first_h;
+        int next_n = 0;      // next item of the CTA's sequence (not yet looked at)
+        int n = -1;          // current item
         int x = 1;           // current row tile of the item
         uint32_t uses = 0;   // units (item, row tile) this slot has computed
-        uint32_t items = 0;  // items this slot has looked at
         int f0 = 0, L = 0, hcur = 0, nkeys = 16, s = 0, sv = 0;
         bool ok = true;
 
@@ -345,36 +292,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the current phase or the one after it).
         auto advance = [&]() -> bool {
             if (!(x == 0 && L > kQTile)) {
-                n += 2;
-                s = n % p.sqk;
-                sv = n % p.nsv;
-                if (leader) {
-                    if (!wait_bar(smem_u32(&bars->qk_full[s]), (uint32_t)(n / p.sqk) & 1, abort_flag, wait_ns,
-                                  p.status)) {
-                        ok = false;
+                // the slot's next item: pass over the other slot's one
+                for (;;) {
+                    int sf0, sL, sseq;
+                    if (!w.find(b, lane, sf0, sL, sseq))
                         return false;
+                    const int nn = next_n++;
+                    const int hh = h;
+                    b += step_b;
+                    h += step_h;
+                    if (h >= H) {
+                        h -= H;
+                        ++b;
                     }
-                    if (lane == 0)
-                        mbar_arrive(smem_u32(&bars->desc_ready[t]));
-                } else if (!wait_bar(smem_u32(&bars->desc_ready[t]), items & 1, abort_flag, wait_ns, p.status)) {
-                    ok = false;
-                    return false;
+                    if ((nn & 1) != t)
+                        continue;
+                    n = nn;
+                    f0 = sf0;
+                    L = sL;
+                    hcur = hh;
+                    break;
                 }
-                ++items;
-                const ItemDesc d = bars->desc[n % kDescRing];
-                if (d.L < 0)
-                    return false;
-                f0 = d.f0;
-                L = d.L;
-                hcur = d.h;
                 x = 0;
                 nkeys = (L + 15) & ~15;   // MMA extent over keys
+                s = n % p.sqk;
+                sv = n % p.nsv;
             } else {
                 x = 1;
             }
             if (leader) {
                 if (lane == 0)
                     NLE_TRACE_AT(1 + t, n * 2 + x, 0);
+                if (x == 0 &&
+                    !wait_bar(smem_u32(&bars->qk_full[s]), (uint32_t)(n / p.sqk) & 1, abort_flag, wait_ns, p.status)) {
+                    ok = false;
+                    return false;
+                }
                 if (uses > 0 &&
                     !wait_bar(smem_u32(&bars->wg_o[t]), (uses - 1) & 1, abort_flag, wait_ns, p.status)) {
                     ok = false;
@@ -411,33 +364,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok)
                 break;
             if (pending) {
-                // Stage 16 rows at a time in shared memory, then write them
-                // with warp-contiguous stores: each store instruction covers
-                // four whole 128-byte rows.  Rows past the block end are
-                // never written.
-                const int rows_left = eL - erow0;   // valid rows of this warp (> 0)
-                __nv_bfloat16 *obase = p.out + (size_t)(ef0 + erow0) * p.out_stride + eh * 64;
+                // rows past the block end are never written
+                if (erow0 + lane < eL) {
+                    uint4 *dst =
+                        reinterpret_cast<uint4 *>(p.out + (size_t)(ef0 + erow0 + lane) * p.out_stride + eh * 64);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    if (half * 16 < rows_left) {
-                        if ((lane >> 4) == half) {
-                            const int r = lane & 15;
-#pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                *reinterpret_cast<uint4 *>(stage + r * 128 + ((c ^ (r & 7)) << 4)) =
-                                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                        }
-                        __syncwarp();
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int r = 4 * i + (lane >> 3), c = lane & 7;
-                            if (half * 16 + r < rows_left) {
-                                const uint4 val = *reinterpret_cast<const uint4 *>(stage + r * 128 + ((c ^ (r & 7)) << 4));
-                                *reinterpret_cast<uint4 *>(obase + (size_t)(half * 16 + r) * p.out_stride + c * 8) = val;
-                            }
-                        }
-                        __syncwarp();
-                    }
+                    for (int c = 0; c < 8; ++c)
+                        dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                 }
                 pending = false;
             }
@@ -490,12 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // rows advance the start address by 2048 bytes.
                 const uint64_t dv = smem_desc_sw128(v_base + sv * p.v_bytes, 0, 1024);
                 if (elect_one()) {
-                    const int ksteps = nkeys / 16;
-#pragma unroll
-                    for (int kk = 0; kk < NB / 16; ++kk)
-                        if (kk < ksteps)
-                            mma_ts(slot + kOCol, slot + kk * 8, dv + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
-                                   kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < nkeys / 16; ++kk)
+                        mma_ts(slot + kOCol, slot + kk * 8, dv + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
+                               kk > 0 ? 1u : 0u);
                     mma_commit(smem_u32(&bars->o_full[t]));
                     if (x == 1 || L <= kQTile)   // the item's last PV: its V stage can be reused
                         mma_commit(smem_u32(&bars->v_empty[sv]));
@@ -512,16 +442,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (active) {
                 uint32_t o[64];
 #pragma unroll
-                for (int c = 0; c < 64; c += 32)
-                    tmem_ld32_nowait(tS + kOCol + c, &o[c]);
+                for (int c = 0; c < 64; c += 16)
+                    tmem_ld16_nowait(tS + kOCol + c, &o[c]);
                 tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    reg_fence(o[i]);
                 const float inv = 1.f / l;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    reg_fence(o[2 * i]);
-                    reg_fence(o[2 * i + 1]);
+                for (int i = 0; i < 32; ++i)
                     pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-                }
             }
             tc_fence_before();
             __syncwarp();
@@ -643,10 +573,7 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
     // tile warpgroups take alternate items, so each stage then belongs to
     // one warpgroup), as deep as fits (V first: it is held from the item's
     // first PV to its last), then the barriers and alignment slack.
-    // barriers and descriptors, then 2 KB of output staging per tile warp,
-    // then slack for aligning the base to 1024 bytes
-    const size_t bars_round = ((sizeof(Bars) + 127) / 128) * 128;
-    const size_t bars_bytes = bars_round + kStageBytes + 1024;
+    const size_t bars_bytes = ((sizeof(Bars) + 127) / 128) * 128 + 1024;
     int sqk = 0, nsv = 0;
     for (const int v : {4, 2}) {
         for (const int q : {4, 2})
@@ -663,7 +590,6 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
     p.sqk = sqk;
     p.nsv = nsv;
     p.bars_off = (uint32_t)(sqk * p.qk_bytes + nsv * p.v_bytes);
-    p.stage_off = p.bars_off + (uint32_t)bars_round;
     const size_t fixed = (size_t)nsv * p.v_bytes + bars_bytes;
     size_t smem = (size_t)sqk * p.qk_bytes + fixed;
     // One CTA per SM: it owns all 512 TMEM columns, so a second resident CTA

@@ -292,7 +292,6 @@ struct PlanWalker {
     int n_seq;
     int total;
     int unit;
-    int mode;       // units enumerated: 0 every unit, 1 only whole units, 2 only each utterance's partial last unit
     int base;       // first utterance of the current group of 32
     int before;     // units in utterances [0, base)
     int incl;       // this lane's inclusive prefix of units within the group
@@ -313,8 +312,7 @@ struct PlanWalker {
                 flag = 1;
                 a = b = 0;
             } else {
-                const int whole = (b - a) / unit, part = (b - a) % unit != 0;
-                n = mode == 0 ? whole + part : (mode == 1 ? whole : part);
+                n = (b - a + unit - 1) / unit;
             }
         }
         start = a;
@@ -333,14 +331,12 @@ struct PlanWalker {
             bad = 1;
     }
 
-    __device__ __forceinline__ void init(const int32_t *cu_, int n_seq_, int total_, int unit_, int lane,
-                                         int mode_ = 0)
+    __device__ __forceinline__ void init(const int32_t *cu_, int n_seq_, int total_, int unit_, int lane)
     {
         cu = cu_;
         n_seq = n_seq_;
         total = total_;
         unit = unit_;
-        mode = mode_;
         base = 0;
         before = 0;
         bad = 0;
@@ -365,55 +361,11 @@ struct PlanWalker {
         const int st = __shfl_sync(kFull, start, src);
         const int ln = __shfl_sync(kFull, len, src);
         const int nb = __shfl_sync(kFull, units, src);
-        const int j = mode == 2 ? ln / unit : rel - (incl_s - nb);   // unit index inside the utterance
+        const int j = rel - (incl_s - nb);
         frame0 = st + j * unit;
         L = min(unit, ln - j * unit);
         seq = base + src;
         return true;
-    }
-};
-
-// The blocks of a packed batch with every whole block first (in batch
-// order) and then every utterance's partial last block (in batch order): a
-// persistent kernel that deals items round-robin then gives each CTA the
-// same mix of large items first and the small ones last, which evens out
-// the CTAs' total work.  Warp-cooperative like PlanWalker; init counts the
-// whole blocks of the batch (one pass over cu_seqlens).
-struct WholeFirstWalker {
-    PlanWalker w;
-    long long n_whole;
-    bool second;
-    int bad;
-
-    __device__ __forceinline__ void init(const int32_t *cu, int n_seq, int total, int unit, int lane)
-    {
-        long long c = 0;
-#pragma unroll 4
-        for (int s = lane; s < n_seq; s += 32) {
-            const int a = __ldg(cu + s), b = __ldg(cu + s + 1);
-            if (a >= 0 && b >= a && b <= total)
-                c += (b - a) / unit;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            c += __shfl_xor_sync(kFull, c, o);
-        n_whole = c;
-        second = false;
-        bad = 0;
-        w.init(cu, n_seq, total, unit, lane, 1);
-    }
-
-    // Locate block u of this order (u non-decreasing over the calls).
-    __device__ __forceinline__ bool find(long long u, int lane, int &frame0, int &L, int &seq)
-    {
-        if (!second && u >= n_whole) {
-            bad |= w.bad;
-            w.init(w.cu, w.n_seq, w.total, w.unit, lane, 2);
-            second = true;
-        }
-        const bool ok = w.find(second ? u - n_whole : u, lane, frame0, L, seq);
-        bad |= w.bad;
-        return ok;
     }
 };
 

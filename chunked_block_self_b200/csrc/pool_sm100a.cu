@@ -331,6 +331,7 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_kernel(PoolParams
 // them.  The arithmetic is the one of posterior_pool_kernel.
 constexpr int kPipe = 3;       // windows in flight per warp
 constexpr int kPipeMaxP = 4;   // frames per window on this path
+constexpr uint32_t kPipeHdr = (kPipe * sizeof(int2) + 15) / 16 * 16;   // slot headers, padded to 16 bytes
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
 {
@@ -345,28 +346,32 @@ __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolParams p, long long per_warp,
-                                                                          uint32_t slot_bytes)
+__global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolParams p, uint32_t slot_bytes)
 {
     extern __shared__ __align__(16) uint8_t pool_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint8_t *ring = pool_smem + (size_t)warp * (kPipe * slot_bytes + kPipe * sizeof(int2));
+    // per warp: kPipe slots, then the slots' headers; slot_bytes and the
+    // header block are multiples of 16, so every cp.async destination is
+    // 16-byte aligned
+    uint8_t *ring = pool_smem + (size_t)warp * (kPipe * slot_bytes + kPipeHdr);
     int2 *hdr = reinterpret_cast<int2 *>(ring + kPipe * slot_bytes);
     const int n_chunks = p.dim >> 3, z_chunks = p.n_classes >> 3;
     const uint32_t hid_bytes = (uint32_t)(p.P * p.dim * 2);   // a slot: P hidden rows, then P logit rows
+    // windows gw, gw + stride, ...: at any moment the warps of the grid work
+    // on neighbouring windows (DRAM pages shared), each keeping kPipe of its
+    // own in flight
     const long long gw = (long long)blockIdx.x * kPoolWarps + warp;
-    const long long g0 = gw * per_warp;
-    const long long g1 = g0 + per_warp < p.n_rows ? g0 + per_warp : p.n_rows;
-    if (g0 >= g1)
+    const long long stride = (long long)gridDim.x * kPoolWarps;
+    if (gw >= p.n_rows)
         return;
     PlanWalker w;
     w.init(p.cu, p.n_seq, p.total, p.P, lane);
-    long long next = g0;   // next window whose copies are issued
+    long long next = gw;   // next window whose copies are issued
     bool more = true;
     // copies of window `next` into slot s (or an end mark), as one group
     auto issue = [&](int s) {
         int f0 = 0, L = -1, seq;
-        if (more && next < g1 && w.find(next, lane, f0, L, seq)) {
+        if (more && next < p.n_rows && w.find(next, lane, f0, L, seq)) {
             uint8_t *slot = ring + (size_t)s * slot_bytes;
             for (int t = 0; t < L; ++t) {
                 const __nv_bfloat16 *hrow = p.hidden + (long long)(f0 + t) * p.h_stride;
@@ -382,21 +387,23 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolP
         }
         if (lane == 0)
             hdr[s] = make_int2(f0, L);
-        ++next;
+        next += stride;
         cp_async_commit();
     };
 #pragma unroll
     for (int s = 0; s < kPipe - 1; ++s)
         issue(s);
-    for (long long g = g0; g < g1; ++g) {
-        const int s = (int)((g - g0) % kPipe);
-        issue((s + kPipe - 1) % kPipe);   // window g + kPipe - 1, into the slot freed last pass
+    long long last = -1;   // the last window this warp pooled
+    for (long long g = gw, k = 0; g < p.n_rows; g += stride, ++k) {
+        const int s = (int)(k % kPipe);
+        issue((s + kPipe - 1) % kPipe);   // this warp's window k + kPipe - 1, into the slot freed last pass
         cp_async_wait<kPipe - 1>();       // this lane's copies of window g have landed
         __syncwarp();
         const int2 hd = hdr[s];
         if (hd.y < 0)
             break;   // past the batch's last window
         const int f0 = hd.x, L = hd.y;
+        last = g;
         const uint8_t *slot = ring + (size_t)s * slot_bytes;
         float lw[kPipeMaxP];
         float M = -INFINITY;
@@ -444,10 +451,10 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolP
         __syncwarp();   // slot s is refilled by the next pass
     }
     cp_async_wait<0>();
-    // the warp holding the last pooled row checks that the batch has no
+    // the warp that pooled row n_rows - 1 checks that the batch has no
     // further window (more windows than rows: nothing past the buffer is
     // written, the shortfall is reported)
-    if (g1 == p.n_rows) {
+    if (last == p.n_rows - 1) {
         int a, b, c;
         if (w.find(p.n_rows, lane, a, b, c) && lane == 0)
             report(p.status, NLE_ERR_INVALID_ARG);
@@ -503,19 +510,18 @@ extern "C" int nle_posterior_pool_fwd(const void *hidden, int64_t hidden_stride,
     const bool vec = (reinterpret_cast<uintptr_t>(logits) & 15) == 0 && logits_stride % 8 == 0 && n_classes % 8 == 0;
     if (vec && n_classes <= 256 && dim <= 1024 && pool_frames <= kPipeMaxP) {
         const uint32_t slot = (uint32_t)(pool_frames * (dim + n_classes) * 2);
-        const size_t smem_cta = (size_t)kPoolWarps * (kPipe * slot + kPipe * sizeof(int2));
+        const size_t smem_cta = (size_t)kPoolWarps * (kPipe * slot + kPipeHdr);
         int per_sm = (int)((200u * 1024u) / smem_cta);
         per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
         long long warps = (long long)di.sm_count * per_sm * kPoolWarps;
         if (warps > n_pooled_rows)
             warps = n_pooled_rows;
-        const long long per_warp = (n_pooled_rows + warps - 1) / warps;
         const long long ctas = (warps + kPoolWarps - 1) / kPoolWarps;
         if (smem_cta > 48 * 1024 && !nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(posterior_pool_pipe_kernel),
                                                                  dev, di.smem_optin))
             return NLE_ERR_CUDA;
         posterior_pool_pipe_kernel<<<(int)ctas, kPoolThreads, smem_cta, static_cast<cudaStream_t>(stream)>>>(
-            p, per_warp, slot);
+            p, slot);
         return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
     }
     // per-warp log weights of a window: above 48 KB (pool_frames > 3072)

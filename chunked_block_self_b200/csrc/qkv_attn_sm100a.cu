@@ -27,21 +27,26 @@
 //               N=192, K=16 x 4 per stage, fp32 accumulator in TMEM
 //               columns 0..191.
 //   warps 4-7   projection epilogue: per row (TMEM lane) reads D, adds the
-//               bias, rounds to bf16 and writes the row's q, k and v into
-//               shared memory in the layouts the attention MMAs read (Q and
-//               K K-major, V N-major, 128-byte swizzle); rows at or past the
-//               block end are written as zeros.  Then D is released for the
-//               next row tile's projection.
+//               bias (fetched into shared memory when the item starts),
+//               rounds to bf16 and writes the row's q into TMEM (columns
+//               192 + 32 x, bf16 pairs: the A operand of the S MMA) and its k
+//               and v into shared memory in the layouts the attention MMAs
+//               read (K K-major, V N-major, 128-byte swizzle); rows at or
+//               past the block end are written as zeros.  Then D is released
+//               for the next row tile's projection.
 //   warps 8-11  attention, as one tile warpgroup of the block kernel, on
-//               TMEM columns 256..511: S = Q_x K^T (M=128, N=ceil16(L)),
-//               fp32 register softmax with one shift per row, P (bf16) over
-//               S, O = P V (P from TMEM), O / rowsum rounded to bf16 and
-//               written with warp-contiguous stores through a small staging
-//               buffer; rows past the block end are never written.
+//               TMEM columns 256..511: S = Q_x K^T (M=128, N=ceil16(L), A
+//               from TMEM), fp32 register softmax with one shift per row, P
+//               (bf16) over S, O = P V (P from TMEM), O / rowsum rounded to
+//               bf16 and written with 16-byte stores; rows past the block
+//               end are never written.
 // The projection of the next item runs in its own TMEM columns while the
-// current item's attention runs; the epilogue of the next item's first row
-// tile waits until the current item's last attention MMA has completed
-// (one set of Q/K/V buffers).
+// current item's attention runs.  There is one set of Q/K/V buffers: the
+// epilogue of the next item's first row tile stores Q and K once the current
+// item's last S MMA has completed, holds V in registers and releases D (so
+// the next row tile's projection starts), and stores V once the current
+// item's last PV has completed.  With Q in TMEM, shared memory holds K, V
+// and four 40 KB stages (B <= 256).
 //
 // Every mbarrier wait is bounded (see nle_device.cuh); on expiry the CTA
 // drains its copies and MMAs in flight, frees TMEM and returns.
@@ -51,6 +56,26 @@
 #include "attn_softmax.cuh"
 #include "nle_device.cuh"
 #include "nle_host.h"
+
+// Optional cycle trace of CTA 0 for performance analysis (not built by
+// default): QKV_TRACE_AT(role, item, event) stores clock64() into a device
+// buffer registered with nle_qkv_trace_set().
+#ifdef NLE_TRACE
+__device__ unsigned long long *g_qkv_trace = nullptr;
+extern "C" int nle_qkv_trace_set(void *p)
+{
+    return cudaMemcpyToSymbol(g_qkv_trace, &p, sizeof(p)) == cudaSuccess ? 0 : -1;
+}
+#define QKV_TRACE_AT(role, n, ev)                                                                       \
+    do {                                                                                                \
+        if (blockIdx.x == 0 && g_qkv_trace && (n) < 64)                                                 \
+            g_qkv_trace[((role) * 64 + (n)) * 16 + (ev)] = clock64();                                   \
+    } while (0)
+#else
+#define QKV_TRACE_AT(role, n, ev) \
+    do {                          \
+    } while (0)
+#endif
 
 namespace {
 
@@ -72,7 +97,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kDCol = 0;      // projection accumulator, 192 columns
 constexpr uint32_t kSCol = 256;    // attention: S (<= 256 columns), P over S, O at +128
 constexpr uint32_t kOCol = 128;
-constexpr uint32_t kOutStage = 4 * 2048;         // output staging: 2 KB per attention warp
+constexpr uint32_t kQCol = 192;    // Q of row tile x (bf16 pairs, 32 columns) at 192 + 32 x
 
 struct ItemDesc {
     int f0, L, h, pad;
@@ -84,12 +109,14 @@ struct Bars {
     uint64_t d_full;                 // the row tile's projection has completed
     uint64_t d_empty;                // 4 arrivals: the epilogue has read D
     uint64_t qkv_ready;              // 4 arrivals: the item's Q, K, V are in shared memory
-    uint64_t qkv_free;               // the item's last attention MMA has completed
+    uint64_t qk_free;                // the item's last S MMA has completed (Q and K read)
+    uint64_t v_free;                 // the item's last PV MMA has completed (V read)
     uint64_t desc_full[kDescRing];
     uint64_t desc_empty[kDescRing];  // every reader has read the entry
     uint64_t s_full, wg_p, o_full, wg_o;
     uint64_t mma_done[2];
     ItemDesc desc[kDescRing];
+    uint4 bias[4][24];               // the current item's 192 bias values, one copy per epilogue warp
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -102,8 +129,7 @@ struct Params {
     int B;            // block_frames
     int ksteps;       // input features / 64
     int nst;          // stage ring depth
-    int qrows;        // rows of the Q buffer (max(NB, 128))
-    uint32_t k_off, v_off, st_off, bars_off, ostage_off;
+    uint32_t v_off, st_off, bars_off;   // K at 0, then V, stages, barriers
     const __nv_bfloat16 *bias;   // nullable, [3 * heads * 64]
     float scale_log2;
     __nv_bfloat16 *out;
@@ -128,13 +154,10 @@ __device__ __forceinline__ uint64_t policy_evict_normal()
 }
 
 // 64 fp32 accumulator columns of this lane's row (+ bias), rounded to bf16
-// and stored as one 128-byte row of a 128-byte-swizzled operand buffer (the
-// 16-byte chunk c of row r sits at chunk position c ^ (r & 7)); zeros when
-// the row lies at or past the block end; nothing stored when `store` is
-// false.  The TMEM loads are warp-collective: every lane of the warp calls
-// this, whatever its row.
-__device__ __forceinline__ void epi_part(uint32_t taddr, const __nv_bfloat16 *bias, bool valid, bool store,
-                                         uint8_t *row_dst, int r)
+// pairs in `pk` (zeros when the row lies at or past the block end).  The
+// TMEM loads are warp-collective: every lane of the warp calls this,
+// whatever its row.
+__device__ __forceinline__ void epi_load(uint32_t taddr, const uint4 *bias, bool valid, uint32_t (&pk)[32])
 {
     uint32_t v[64];
     tmem_ld32_nowait(taddr, &v[0]);
@@ -147,7 +170,7 @@ __device__ __forceinline__ void epi_part(uint32_t taddr, const __nv_bfloat16 *bi
     for (int c = 0; c < 8; ++c) {
         float b[8];
         if (bias) {
-            const uint4 bw = __ldg(reinterpret_cast<const uint4 *>(bias) + c);
+            const uint4 bw = bias[c];
             const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -159,20 +182,22 @@ __device__ __forceinline__ void epi_part(uint32_t taddr, const __nv_bfloat16 *bi
             for (int e = 0; e < 8; ++e)
                 b[e] = 0.f;
         }
-        uint4 q = make_uint4(0, 0, 0, 0);
-        if (valid) {
-            float f[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                f[e] = __uint_as_float(v[8 * c + e]) + b[e];
-            q.x = pack_bf16x2(f[0], f[1]);
-            q.y = pack_bf16x2(f[2], f[3]);
-            q.z = pack_bf16x2(f[4], f[5]);
-            q.w = pack_bf16x2(f[6], f[7]);
-        }
-        if (store)
-            *reinterpret_cast<uint4 *>(row_dst + ((c ^ (r & 7)) << 4)) = q;
+        for (int e = 0; e < 4; ++e)
+            pk[4 * c + e] = valid ? pack_bf16x2(__uint_as_float(v[8 * c + 2 * e]) + b[2 * e],
+                                                __uint_as_float(v[8 * c + 2 * e + 1]) + b[2 * e + 1])
+                                  : 0u;
     }
+}
+
+// One 128-byte row of a 128-byte-swizzled operand buffer: the 16-byte chunk
+// c of row r sits at chunk position c ^ (r & 7).
+__device__ __forceinline__ void epi_store(const uint32_t (&pk)[32], uint8_t *row_dst, int r)
+{
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4 *>(row_dst + ((c ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
 }
 
 template <int NB>
@@ -182,10 +207,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t q_base = smem_u32(smem);
-    const uint32_t k_base = q_base + p.k_off;
-    const uint32_t v_base = q_base + p.v_off;
-    const uint32_t st_base = q_base + p.st_off;
+    const uint32_t k_base = smem_u32(smem);
+    const uint32_t v_base = k_base + p.v_off;
+    const uint32_t st_base = k_base + p.st_off;
     Bars *bars = reinterpret_cast<Bars *>(smem + p.bars_off);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -199,7 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(&bars->d_full), 1);
         mbar_init(smem_u32(&bars->d_empty), 4);
         mbar_init(smem_u32(&bars->qkv_ready), 4);
-        mbar_init(smem_u32(&bars->qkv_free), 1);
+        mbar_init(smem_u32(&bars->qk_free), 1);
+        mbar_init(smem_u32(&bars->v_free), 1);
         for (int j = 0; j < kDescRing; ++j) {
             mbar_init(smem_u32(&bars->desc_full[j]), 1);
             mbar_init(smem_u32(&bars->desc_empty[j]), kDescReaders);
@@ -274,6 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             const int tiles = L > kQTile ? 2 : 1;
+            if (lane == 0)
+                QKV_TRACE_AT(0, n, 0);
             for (int x = 0; x < tiles && ok; ++x) {
                 for (int kb = 0; kb < KS; ++kb, ++g) {
                     const int s = (int)(g % (uint32_t)p.nst);
@@ -290,6 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d(dst + kXBytes, &tm_w, kb * 64, h * 64, bar, pol_w);
                         tma_load_2d(dst + kXBytes + 8192, &tm_w, kb * 64, (H + h) * 64, bar, pol_w);
                         tma_load_2d(dst + kXBytes + 16384, &tm_w, kb * 64, (2 * H + h) * 64, bar, pol_w);
+                        if (kb == 0)
+                            QKV_TRACE_AT(0, n, 1 + x);
+                        if (kb == KS - 1)
+                            QKV_TRACE_AT(0, n, 3 + x);
                     }
                     __syncwarp();
                 }
@@ -332,6 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
+                if (lane == 0)
+                    QKV_TRACE_AT(1, n, 3 * x);
                 for (int kb = 0; kb < KS; ++kb, ++g) {
                     const int s = (int)(g % (uint32_t)p.nst);
                     if (!wait_bar(smem_u32(&bars->st_full[s]), (g / (uint32_t)p.nst) & 1, abort_flag, wait_ns,
@@ -339,6 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (lane == 0 && kb == 0)
+                        QKV_TRACE_AT(1, n, 3 * x + 1);
                     tc_fence_after();
                     const uint32_t a = st_base + (uint32_t)s * kStageBytes;
                     const uint64_t da = smem_desc_sw128(a, 16, 1024);
@@ -348,8 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int kk = 0; kk < 4; ++kk)
                             mma_ss(tmem + kDCol, da + 2 * kk, db + 2 * kk, id_p, (kb | kk) ? 1u : 0u);
                         mma_commit(smem_u32(&bars->st_empty[s]));
-                        if (kb == KS - 1)
+                        if (kb == KS - 1) {
                             mma_commit(smem_u32(&bars->d_full));
+                            QKV_TRACE_AT(1, n, 3 * x + 2);
+                        }
                     }
                     __syncwarp();
                 }
@@ -367,12 +404,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ==================================================== projection epilogue
         const int qq = warp & 3;
         const uint32_t tD = tmem + kDCol + ((uint32_t)(qq * 32) << 16);
+        const uint32_t tQ = tmem + kQCol + ((uint32_t)(qq * 32) << 16);
         const int NBr = ((p.B + 15) / 16) * 16;   // K and V rows the attention MMAs may read
+        uint4 *wbias = bars->bias[qq];
         uint32_t tiles_done = 0;
         for (int n = 0;; ++n) {
             ItemDesc d;
             if (!read_desc(n, d) || d.L < 0)
                 break;
+            // this item's q, k and v bias rows, fetched while its projection
+            // runs (off the path from the finished projection to the release
+            // of D)
+            if (p.bias && lane < 24)
+                wbias[lane] = __ldg(reinterpret_cast<const uint4 *>(p.bias + (size_t)((lane >> 3) * H + d.h) * 64) +
+                                    (lane & 7));
+            __syncwarp();
+            const uint4 *bq = p.bias ? wbias : nullptr;
+            const uint4 *bk = p.bias ? wbias + 8 : nullptr;
+            const uint4 *bv = p.bias ? wbias + 16 : nullptr;
             const int tiles = d.L > kQTile ? 2 : 1;
             bool ok = true;
             for (int x = 0; x < tiles; ++x) {
@@ -380,31 +429,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                // the previous item's attention must be done with Q, K and V
-                if (x == 0 && n > 0 &&
-                    !wait_bar(smem_u32(&bars->qkv_free), (uint32_t)(n - 1) & 1, abort_flag, wait_ns, p.status)) {
+                tc_fence_after();
+                if (warp == kEpi0 && lane == 0)
+                    QKV_TRACE_AT(2, n, 5 * x);
+                const int r = x * kQTile + qq * 32 + lane;   // block row of this lane
+                const bool valid = r < d.L;
+                // every lane runs the (warp-collective) TMEM loads and
+                // stores; only rows inside the buffers are stored to shared
+                // memory.  The previous item's attention still reads the
+                // buffers: Q (TMEM columns 192..255) and K until its last S
+                // MMA has completed, V until its last PV.  V is held in
+                // registers meanwhile, so D is released for the next row
+                // tile's projection without waiting for that PV.
+                const bool first_tile_of_later_item = x == 0 && n > 0;
+                if (first_tile_of_later_item &&
+                    !wait_bar(smem_u32(&bars->qk_free), (uint32_t)(n - 1) & 1, abort_flag, wait_ns, p.status)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                const int r = x * kQTile + qq * 32 + lane;   // block row of this lane
-                const bool valid = r < d.L;
-                const __nv_bfloat16 *bq = p.bias ? p.bias + (size_t)d.h * 64 : nullptr;
-                const __nv_bfloat16 *bk = p.bias ? p.bias + (size_t)(H + d.h) * 64 : nullptr;
-                const __nv_bfloat16 *bv = p.bias ? p.bias + (size_t)(2 * H + d.h) * 64 : nullptr;
-                // every lane runs the (warp-collective) TMEM loads; only
-                // rows inside the buffers are stored
-                epi_part(tD, bq, valid, r < p.qrows, smem + (size_t)r * kRowBytes, r);
-                epi_part(tD + 64, bk, valid, r < NBr, smem + p.k_off + (size_t)r * kRowBytes, r);
-                epi_part(tD + 128, bv, valid, r < NBr, smem + p.v_off + (size_t)r * kRowBytes, r);
-                fence_proxy_async_smem();   // the rows are read by the async proxy (MMAs)
+                if (warp == kEpi0 && lane == 0)
+                    QKV_TRACE_AT(2, n, 5 * x + 1);
+                {
+                    uint32_t pk[32];
+                    epi_load(tD, bq, valid, pk);
+                    tmem_st32(tQ + 32 * x, pk);   // Q: the A operand of the S MMA, from TMEM
+                    epi_load(tD + 64, bk, valid, pk);
+                    if (r < NBr)
+                        epi_store(pk, smem + (size_t)r * kRowBytes, r);
+                }
+                uint32_t pv[32];
+                epi_load(tD + 128, bv, valid, pv);
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
+                if (lane == 0)
                     mbar_arrive(smem_u32(&bars->d_empty));
-                    if (x == tiles - 1)
-                        mbar_arrive(smem_u32(&bars->qkv_ready));
+                if (warp == kEpi0 && lane == 0)
+                    QKV_TRACE_AT(2, n, 5 * x + 2);
+                if (first_tile_of_later_item &&
+                    !wait_bar(smem_u32(&bars->v_free), (uint32_t)(n - 1) & 1, abort_flag, wait_ns, p.status)) {
+                    ok = false;
+                    break;
                 }
+                if (warp == kEpi0 && lane == 0)
+                    QKV_TRACE_AT(2, n, 5 * x + 3);
+                if (r < NBr)
+                    epi_store(pv, smem + p.v_off + (size_t)r * kRowBytes, r);
+                fence_proxy_async_smem();   // the rows are read by the async proxy (MMAs)
+                __syncwarp();
+                if (lane == 0 && x == tiles - 1)
+                    mbar_arrive(smem_u32(&bars->qkv_ready));
+                if (warp == kEpi0 && lane == 0)
+                    QKV_TRACE_AT(2, n, 5 * x + 4);
                 ++tiles_done;
             }
             if (!ok)
@@ -418,7 +494,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tS = slot + ((uint32_t)(qq * 32) << 16);
         const float sl2 = p.scale_log2;
         const uint32_t id_pv = idesc_bf16_f32(128, 64, true);
-        uint8_t *stage = smem + p.ostage_off + (uint32_t)qq * 2048u;
         int n = -1, x = 1, L = 0, f0 = 0, hcur = 0, nkeys = 16;
         uint32_t uses = 0;
         bool ok = true;
@@ -455,14 +530,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     return false;
                 }
                 tc_fence_after();
-                const uint64_t da = smem_desc_sw128(q_base + (uint32_t)(x * kQTile * kRowBytes), 16, 1024);
+                if (lane == 0)
+                    QKV_TRACE_AT(3, n, 4 * x);
+                // A = Q of the row tile from TMEM (K = 64 in 4 steps of 8
+                // columns of bf16 pairs), B = K from shared memory
+                const uint32_t qa = tmem + kQCol + (uint32_t)(32 * x);
                 const uint64_t db = smem_desc_sw128(k_base, 16, 1024);
                 const uint32_t id_s = idesc_bf16_f32(128, nkeys, false);
                 if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(slot, da + 2 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
+                        mma_ts(slot, qa + 8 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
                     mma_commit(smem_u32(&bars->s_full));
+                    if (x == 1 || L <= kQTile)   // the item's last S: Q and K may be overwritten
+                        mma_commit(smem_u32(&bars->qk_free));
                 }
                 __syncwarp();
             }
@@ -477,34 +558,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok)
                 break;
             if (pending) {
-                // 16 rows at a time through the staging buffer, then four
-                // whole 128-byte rows per store instruction; rows past the
-                // block end are never written
-                const int rows_left = eL - erow0;
-                __nv_bfloat16 *obase = p.out + (size_t)(ef0 + erow0) * p.out_stride + eh * 64;
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    if (half * 16 < rows_left) {
-                        if ((lane >> 4) == half) {
-                            const int r = lane & 15;
+                // rows past the block end are never written
+                if (erow0 + lane < eL) {
+                    uint4 *dst =
+                        reinterpret_cast<uint4 *>(p.out + (size_t)(ef0 + erow0 + lane) * p.out_stride + eh * 64);
 #pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                *reinterpret_cast<uint4 *>(stage + r * 128 + ((c ^ (r & 7)) << 4)) =
-                                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                        }
-                        __syncwarp();
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int r = 4 * i + (lane >> 3), c = lane & 7;
-                            if (half * 16 + r < rows_left) {
-                                const uint4 val =
-                                    *reinterpret_cast<const uint4 *>(stage + r * 128 + ((c ^ (r & 7)) << 4));
-                                *reinterpret_cast<uint4 *>(obase + (size_t)(half * 16 + r) * p.out_stride + c * 8) =
-                                    val;
-                            }
-                        }
-                        __syncwarp();
-                    }
+                    for (int c = 0; c < 8; ++c)
+                        dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                 }
                 pending = false;
             }
@@ -523,6 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(smem_u32(&bars->wg_p));
+            if (leader && lane == 0)
+                QKV_TRACE_AT(3, n, 4 * x + 1);
             // ---------------------------------------------- O = P V
             if (leader) {
                 if (!wait_bar(smem_u32(&bars->wg_p), uses & 1, abort_flag, wait_ns, p.status))
@@ -538,8 +600,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mma_ts(slot + kOCol, slot + kk * 8, dv + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
                                    kk > 0 ? 1u : 0u);
                     mma_commit(smem_u32(&bars->o_full));
-                    if (x == 1 || L <= kQTile)   // the item's last MMA: Q, K and V may be overwritten
-                        mma_commit(smem_u32(&bars->qkv_free));
+                    QKV_TRACE_AT(3, n, 4 * x + 2);
+                    if (x == 1 || L <= kQTile)   // the item's last PV: V may be overwritten
+                        mma_commit(smem_u32(&bars->v_free));
                 }
                 __syncwarp();
             }
@@ -564,6 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(smem_u32(&bars->wg_o));
+            if (leader && lane == 0)
+                QKV_TRACE_AT(3, n, 4 * x + 3);
             ++uses;
             pending = active;
             ef0 = f0;
@@ -657,17 +722,15 @@ extern "C" int nle_block_attn_qkv_fwd_ex(const void *x, const void *w_qkv, const
     p.heads = heads;
     p.B = B;
     p.ksteps = d_model / 64;
-    // Q holds >= 128 rows (each S MMA reads 128 rows from its tile's base;
-    // row tile 1 reads past the Q rows into the K buffer, rows it ignores)
-    p.qrows = NB > kQTile ? NB : kQTile;
-    const uint32_t q_bytes = (uint32_t)p.qrows * kRowBytes, kv_bytes = (uint32_t)NB * kRowBytes;
-    p.k_off = q_bytes;
-    p.v_off = q_bytes + kv_bytes;
-    p.st_off = (q_bytes + 2 * kv_bytes + 1023) & ~1023u;
+    // shared memory: K and V of the item (NB rows each), the stage ring,
+    // the barriers; Q lives in TMEM
+    const uint32_t kv_bytes = (uint32_t)NB * kRowBytes;
+    p.v_off = kv_bytes;
+    p.st_off = (2 * kv_bytes + 1023) & ~1023u;
     const size_t bars_round = ((sizeof(Bars) + 127) / 128) * 128;
     int nst = 0;
     for (int s = kMaxStages; s >= 2; --s)
-        if ((size_t)p.st_off + (size_t)s * kStageBytes + bars_round + kOutStage + 1024 <= (size_t)di.smem_optin) {
+        if ((size_t)p.st_off + (size_t)s * kStageBytes + bars_round + 1024 <= (size_t)di.smem_optin) {
             nst = s;
             break;
         }
@@ -675,8 +738,7 @@ extern "C" int nle_block_attn_qkv_fwd_ex(const void *x, const void *w_qkv, const
         return NLE_ERR_UNSUPPORTED;
     p.nst = nst;
     p.bars_off = p.st_off + (uint32_t)nst * kStageBytes;
-    p.ostage_off = p.bars_off + (uint32_t)bars_round;
-    size_t smem = (size_t)p.ostage_off + kOutStage + 1024;
+    size_t smem = (size_t)p.bars_off + bars_round + 1024;
     // one CTA per SM: it owns all 512 TMEM columns
     if (smem <= (size_t)di.smem_optin / 2)
         smem = (size_t)di.smem_optin / 2 + 1024;

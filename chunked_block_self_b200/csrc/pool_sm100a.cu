@@ -323,14 +323,17 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_kernel(PoolParams
 
 // ---------------------------------------------------------------- pipelined path
 // For the common shape (windows of at most kPipeMaxP frames, hidden width at
-// most 1024, at most 256 logit classes read as 16-byte chunks) each warp
-// takes a contiguous range of windows and keeps kPipe windows in flight: the
-// frames' hidden rows and logits are copied into a per-warp shared-memory
-// ring with cp.async (16 bytes per lane per copy), so many windows' bytes are
-// on their way from HBM while one is pooled, with no registers held for
-// them.  The arithmetic is the one of posterior_pool_kernel.
-constexpr int kPipe = 3;       // windows in flight per warp
-constexpr int kPipeMaxP = 4;   // frames per window on this path
+// most 1024, at most 256 logit classes read as 16-byte chunks) every warp
+// keeps the next window's bytes in flight while it pools the current one:
+// the frames' hidden rows and logits are copied into a per-warp
+// shared-memory ring with cp.async (16 bytes per lane per copy), with no
+// registers held for them, and the frames' weight reductions run
+// interleaved.  The arithmetic is the one of posterior_pool_kernel.  Small
+// per-warp rings keep up to 20 warps on an SM: the measured time fell from
+// three windows in flight per warp (12 warps per SM) to two (16 warps), and
+// rose with four (8 warps).
+constexpr int kPipe = 2;       // windows in flight per warp
+constexpr int kPipeMaxP = 2;   // frames per window on this path
 constexpr uint32_t kPipeHdr = (kPipe * sizeof(int2) + 15) / 16 * 16;   // slot headers, padded to 16 bytes
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
@@ -344,6 +347,65 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait()
 {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// log(1 - p_blank) of frames t < L of a window (the others -inf), from one
+// 16-byte logit chunk per lane and frame (C <= 256, a multiple of 8): the
+// arithmetic of chunk_log_weight, with the frames' warp reductions
+// interleaved.
+__device__ __forceinline__ void window_log_weights(const uint4 (&q)[kPipeMaxP], int C, int L, int lane,
+                                                   float (&lw)[kPipeMaxP])
+{
+    const bool has = 8 * lane < C;
+    float v[kPipeMaxP][8], m[kPipeMaxP], mnb[kPipeMaxP];
+#pragma unroll
+    for (int t = 0; t < kPipeMaxP; ++t) {
+        chunk_vals(q[t], v[t]);
+        m[t] = -INFINITY;
+        mnb[t] = -INFINITY;
+        if (has && t < L)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                m[t] = fmaxf(m[t], v[t][e]);
+                if (lane > 0 || e > 0)
+                    mnb[t] = fmaxf(mnb[t], v[t][e]);
+            }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int t = 0; t < kPipeMaxP; ++t) {
+            m[t] = fmaxf(m[t], __shfl_xor_sync(kFull, m[t], o));
+            mnb[t] = fmaxf(mnb[t], __shfl_xor_sync(kFull, mnb[t], o));
+        }
+    float sm[kPipeMaxP], snb[kPipeMaxP];
+    bool far[kPipeMaxP];
+#pragma unroll
+    for (int t = 0; t < kPipeMaxP; ++t) {
+        far[t] = mnb[t] - m[t] < -60.f;
+        const float mr = far[t] ? mnb[t] : m[t];
+        sm[t] = 0.f;
+        snb[t] = 0.f;
+        if (has && t < L && mnb[t] != -INFINITY)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float x = exp2f((v[t][e] - m[t]) * kLog2e);
+                sm[t] += x;
+                if (lane > 0 || e > 0)
+                    snb[t] += far[t] ? exp2f((v[t][e] - mr) * kLog2e) : x;
+            }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int t = 0; t < kPipeMaxP; ++t) {
+            sm[t] += __shfl_xor_sync(kFull, sm[t], o);
+            snb[t] += __shfl_xor_sync(kFull, snb[t], o);
+        }
+#pragma unroll
+    for (int t = 0; t < kPipeMaxP; ++t)
+        lw[t] = (t < L && mnb[t] != -INFINITY) ? (far[t] ? mnb[t] - m[t] : 0.f) + (logf(snb[t]) - logf(sm[t]))
+                                              : -INFINITY;
 }
 
 __global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolParams p, uint32_t slot_bytes)
@@ -405,16 +467,19 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolP
         const int f0 = hd.x, L = hd.y;
         last = g;
         const uint8_t *slot = ring + (size_t)s * slot_bytes;
+        uint4 zq[kPipeMaxP];
+#pragma unroll
+        for (int t = 0; t < kPipeMaxP; ++t) {
+            zq[t] = make_uint4(0u, 0u, 0u, 0u);
+            if (t < L && lane < z_chunks)
+                zq[t] = *reinterpret_cast<const uint4 *>(slot + hid_bytes + (size_t)(t * p.n_classes + 8 * lane) * 2);
+        }
         float lw[kPipeMaxP];
+        window_log_weights(zq, p.n_classes, L, lane, lw);
         float M = -INFINITY;
 #pragma unroll
         for (int t = 0; t < kPipeMaxP; ++t) {
-            lw[t] = -INFINITY;
             if (t < L) {
-                uint4 q = make_uint4(0u, 0u, 0u, 0u);
-                if (lane < z_chunks)
-                    q = *reinterpret_cast<const uint4 *>(slot + hid_bytes + (size_t)(t * p.n_classes + 8 * lane) * 2);
-                lw[t] = chunk_log_weight(q, p.n_classes, lane);
                 M = fmaxf(M, lw[t]);
                 if (lane == 0 && p.weights)
                     p.weights[f0 + t] = expf(lw[t]);
@@ -511,8 +576,8 @@ extern "C" int nle_posterior_pool_fwd(const void *hidden, int64_t hidden_stride,
     if (vec && n_classes <= 256 && dim <= 1024 && pool_frames <= kPipeMaxP) {
         const uint32_t slot = (uint32_t)(pool_frames * (dim + n_classes) * 2);
         const size_t smem_cta = (size_t)kPoolWarps * (kPipe * slot + kPipeHdr);
-        int per_sm = (int)((200u * 1024u) / smem_cta);
-        per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+        int per_sm = (int)((size_t)di.smem_optin / (smem_cta + 1024));
+        per_sm = per_sm < 1 ? 1 : (per_sm > 6 ? 6 : per_sm);
         long long warps = (long long)di.sm_count * per_sm * kPoolWarps;
         if (warps > n_pooled_rows)
             warps = n_pooled_rows;

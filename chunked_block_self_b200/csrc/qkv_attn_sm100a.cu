@@ -713,6 +713,8 @@ extern "C" int nle_block_attn_qkv_fwd_ex(const void *x, const void *w_qkv, const
     if (di.cc_major != 10)
         return NLE_ERR_UNSUPPORTED;
 
+    const double scale = softmax_scale > 0.f ? (double)softmax_scale : 1.0 / std::sqrt((double)d_head);
+    const unsigned long long wns = wait_limit_ns > 0 ? (unsigned long long)wait_limit_ns : 1000000000ull;
     const int B = block_frames;
     const int NB = (B + 15) / 16 * 16;
     Params p{};
@@ -743,12 +745,11 @@ extern "C" int nle_block_attn_qkv_fwd_ex(const void *x, const void *w_qkv, const
     if (smem <= (size_t)di.smem_optin / 2)
         smem = (size_t)di.smem_optin / 2 + 1024;
     p.bias = static_cast<const __nv_bfloat16 *>(bias);
-    const double scale = softmax_scale > 0.f ? (double)softmax_scale : 1.0 / std::sqrt((double)d_head);
     p.scale_log2 = (float)(scale * 1.4426950408889634);
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.out_stride = heads * 64;
     p.status = dev_status;
-    p.wait_ns = wait_limit_ns > 0 ? (unsigned long long)wait_limit_ns : 1000000000ull;
+    p.wait_ns = wns;
     p.flags = flags;
 
     CUtensorMap tx, tw;

@@ -59,21 +59,30 @@ NCU_TRAFFIC = {
                    "source_sha256": "4b8b881b30603475fc25697837e89c2228438e3be7aad521f97ca1295d608110",
                    "traffic_over_algorithmic": (378117120 + 66760704) / 482533376,
                    "tensor_pipe_pct": 19.2},
-    "window_xattn": {"files": ("window_xattn_sm100a.cu", "nle_device.cuh"),
-                     "source_sha256": "43ecd044325aac9d122bc38ba666274726781c3720caf2f2a5fcb5b34fb21737",
-                     "traffic_over_algorithmic": (265946112 + 7618304) / 290320384},
+    "window_xattn": {"files": ('window_xattn_sm100a.cu', 'nle_device.cuh'),
+                    "source_sha256": "44c247f038150ebc19ef8299c838232d7615b43f47cd5c35f050e4399dac1c65",
+                    "traffic_over_algorithmic": (265965568 + 7668992) / 290320384},
     # full-utterance attention: the long-clip workload, the same launch as the bench's
-    "varlen_attn": {"files": ("varlen_attn_sm100a.cu", "attn_softmax.cuh", "nle_device.cuh"),
-                    "source_sha256": "f97abe68c26d62ac374fa754a2f1b1536b5e4cc4598e43d5712680b93a44f41f",
-                    "traffic_over_algorithmic": (343228160 + 91153152) / 439304192,
-                    "tensor_pipe_pct": 25.6},
-    "qkv_attn": {"files": ("qkv_attn_sm100a.cu", "attn_softmax.cuh", "nle_device.cuh"),
-                 "source_sha256": "", "traffic_over_algorithmic": None},
+    "varlen_attn": {"files": ('varlen_attn_sm100a.cu', 'attn_softmax.cuh', 'nle_device.cuh'),
+                   "source_sha256": "9f9034f668362301b35d9d87571d4a0718ac495d5026e1ceed7ccc202e3f0714",
+                   "traffic_over_algorithmic": (343928832 + 91376128) / 439304192,
+                   "tensor_pipe_pct": 25.5},
+    # fused projection + block attention on the batch-128 workload (d_model 1024,
+    # 16 heads); DRAM writes sit below the output's bytes because part of it is
+    # still in L2 when the kernel ends
+    "qkv_attn": {"files": ('qkv_attn_sm100a.cu', 'attn_softmax.cuh', 'nle_device.cuh'),
+                 "source_sha256": "2a9ce094c52f98fff402b83e264ef9084cdbfed03fd19d434410850bcb92aff0",
+                 "traffic_over_algorithmic": (127470592 + 82170624) / 247564288,
+                 "tensor_pipe_pct": 44.4},
+    # posterior pooling over the whole batch-128 workload (58,903 frames)
+    "posterior_pool": {"files": ('pool_sm100a.cu', 'nle_device.cuh'),
+                       "source_sha256": "b8d5d604258c92eaf69cbb051ec3912c14a782103b9afa75ecac9a378f4211db",
+                       "traffic_over_algorithmic": (151211776 + 28471552) / 211398236},
     # CTC argmax: captured on 16 utterances (3,300 rows, 662.4 MB); traffic grows
     # with rows, so the ratio is applied to the full batch
-    "ctc_argmax": {"files": ("ctc_sm100a.cu", "nle_device.cuh"),
-                   "source_sha256": "dc0ebd4500f03c2450606136a33502b06bc01edfa47d3ad49651a89a64928637",
-                   "traffic_over_algorithmic": (739271680 + 3598336) / 662369464},
+    "ctc_argmax": {"files": ('ctc_sm100a.cu', 'nle_device.cuh'),
+                  "source_sha256": "02522fcce199cfa9546ef350a028e971b829e49e32cb3e6807e42f62bcfafbd9",
+                  "traffic_over_algorithmic": (662636288 + 3366912) / 662369464},
 }
 
 
@@ -490,7 +499,7 @@ def measure_qkv_attn(nle, dev, stream, reps, rank, lengths, tf_peak):
            "tflops": tflops, "pct_of_dense_bf16_peak": 100.0 * tflops / tf_peak,
            "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_peak, "unit": "TFLOP/s",
                         "frac": tflops / tf_peak, "ai_flop_per_byte": flops / byt},
-           "tensor_pipe_pct": ncu_tensor_pipe_pct("qkv_attn"),
+           "tensor_pipe_pct": ncu_tensor_pipe_pct("qkv_attn"), "traffic": ncu_traffic("qkv_attn", byt),
            "unfused_ms": umed, "unfused_tflops": flops / (umed * 1e-3) / 1e12,
            "unfused": "torch.addmm (cuBLAS) X W^T + b -> Q|K|V in memory, then the block kernel",
            "speedup_vs_unfused": umed / med, "kernels": 1}
@@ -635,7 +644,8 @@ def run_nle(args, rank, world, local):
         pool_bytes = n_fr * (wl.HIDDEN_DIM + wl.CHAR_CLASSES) * 2 + n_rows * wl.HIDDEN_DIM * 2 + n_fr * 4
         pool = {"frames": n_fr, "rows": n_rows, "pool_frames": wl.POOL_FRAMES, "dim": wl.HIDDEN_DIM,
                 "char_classes": wl.CHAR_CLASSES, "ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
-                "algorithmic_bytes": pool_bytes, "l2": "flushed (256 MB write) before each launch", "kernels": 1,
+                "algorithmic_bytes": pool_bytes, "traffic": ncu_traffic("posterior_pool", pool_bytes),
+                "l2": "flushed (256 MB write) before each launch", "kernels": 1,
                 "timing": "median of 50 launches"}
         del px, pooled, pw
 
@@ -700,6 +710,14 @@ def run_nle(args, rank, world, local):
     if not args.no_qkv:
         qkv_att = measure_qkv_attn(nle, dev, stream, args.config_reps, rank, lengths, tf_peak)
     if va is not None:
+        # the exp unit's ceiling: one exp per (query row, key, head) at 16
+        # ex2 results per clock per SM (4 per SM sub-partition), at the SM
+        # clock seen during the timed steps
+        mhz = clocks.summary().get("sm_mhz") or 1965.0
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        exps = va["algorithmic_flops"] / (4 * D)
+        va["exp_ceiling_ms"] = 1e3 * exps / (16 * sms * mhz * 1e6)
+        va["frac_of_exp_ceiling"] = va["exp_ceiling_ms"] / va["ms"]
         va["pct_of_dense_bf16_peak"] = 100.0 * va["tflops"] / tf_peak
         va["roofline"] = {"bound": "tensor", "achieved": va["tflops"], "peak": tf_peak, "unit": "TFLOP/s",
                           "frac": va["tflops"] / tf_peak,

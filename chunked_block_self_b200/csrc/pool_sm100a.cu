@@ -336,6 +336,32 @@ constexpr int kPipe = 2;       // windows in flight per warp
 constexpr int kPipeMaxP = 2;   // frames per window on this path
 constexpr uint32_t kPipeHdr = (kPipe * sizeof(int2) + 15) / 16 * 16;   // slot headers, padded to 16 bytes
 
+// Shared memory of one warp on the pipelined path with NCH hidden chunks
+// per lane: kPipe slots of kPipeMaxP frames, each frame NCH 512-byte rows
+// of hidden chunks (chunk 32 i + lane at row i, column lane) and one of
+// logit chunks, then the slots' headers.
+template <int NCH>
+__host__ __device__ constexpr uint32_t pipe_warp_bytes()
+{
+    return kPipe * kPipeMaxP * (NCH + 1) * 512 + kPipeHdr;
+}
+
+// (d.x, d.y) = (a.x b.x + c.x, a.y b.y + c.y): two fp32 FMAs in one packed
+// instruction, each rounded as fmaf rounds it.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -351,8 +377,12 @@ __device__ __forceinline__ void cp_async_wait()
 
 // log(1 - p_blank) of frames t < L of a window (the others -inf), from one
 // 16-byte logit chunk per lane and frame (C <= 256, a multiple of 8): the
-// arithmetic of chunk_log_weight, with the frames' warp reductions
-// interleaved.
+// arithmetic of chunk_log_weight with the frames' warp reductions
+// interleaved.  Each exponent is one FMA, z log2(e) - m log2(e), and one
+// ex2; the shift's rounding multiplies every term of a frame's two sums by
+// the same factor, which the ratio cancels.  The re-summation about the
+// non-blank maximum (a blank that dominates by more than 60) is a
+// warp-uniform branch of its own.
 __device__ __forceinline__ void window_log_weights(const uint4 (&q)[kPipeMaxP], int C, int L, int lane,
                                                    float (&lw)[kPipeMaxP])
 {
@@ -363,13 +393,12 @@ __device__ __forceinline__ void window_log_weights(const uint4 (&q)[kPipeMaxP], 
         chunk_vals(q[t], v[t]);
         m[t] = -INFINITY;
         mnb[t] = -INFINITY;
-        if (has && t < L)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                m[t] = fmaxf(m[t], v[t][e]);
-                if (lane > 0 || e > 0)
-                    mnb[t] = fmaxf(mnb[t], v[t][e]);
-            }
+        if (has && t < L) {
+            mnb[t] = fmax3(fmax3(v[t][1], v[t][2], v[t][3]), fmax3(v[t][4], v[t][5], v[t][6]), v[t][7]);
+            m[t] = fmaxf(mnb[t], v[t][0]);
+            if (lane > 0)
+                mnb[t] = m[t];
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
@@ -379,20 +408,35 @@ __device__ __forceinline__ void window_log_weights(const uint4 (&q)[kPipeMaxP], 
             mnb[t] = fmaxf(mnb[t], __shfl_xor_sync(kFull, mnb[t], o));
         }
     float sm[kPipeMaxP], snb[kPipeMaxP];
-    bool far[kPipeMaxP];
+    bool far = false;
 #pragma unroll
     for (int t = 0; t < kPipeMaxP; ++t) {
-        far[t] = mnb[t] - m[t] < -60.f;
-        const float mr = far[t] ? mnb[t] : m[t];
         sm[t] = 0.f;
         snb[t] = 0.f;
-        if (has && t < L && mnb[t] != -INFINITY)
+        if (has && t < L && mnb[t] != -INFINITY) {
+            const float ms = m[t] * kLog2e;
+            float x[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float x = exp2f((v[t][e] - m[t]) * kLog2e);
-                sm[t] += x;
-                if (lane > 0 || e > 0)
-                    snb[t] += far[t] ? exp2f((v[t][e] - mr) * kLog2e) : x;
+            for (int e = 0; e < 8; ++e)
+                x[e] = ex2_approx(fmaf(v[t][e], kLog2e, -ms));
+            const float rest = ((x[1] + x[2]) + (x[3] + x[4])) + ((x[5] + x[6]) + x[7]);
+            sm[t] = x[0] + rest;
+            snb[t] = lane > 0 ? sm[t] : rest;
+        }
+        far |= t < L && mnb[t] != -INFINITY && mnb[t] - m[t] < -60.f;
+    }
+    if (far) {   // warp-uniform: m and mnb are the warp's
+#pragma unroll
+        for (int t = 0; t < kPipeMaxP; ++t)
+            if (t < L && mnb[t] != -INFINITY && mnb[t] - m[t] < -60.f) {
+                const float ms = mnb[t] * kLog2e;
+                float acc = 0.f;
+                if (has)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (lane > 0 || e > 0)
+                            acc += ex2_approx(fmaf(v[t][e], kLog2e, -ms));
+                snb[t] = acc;
             }
     }
 #pragma unroll
@@ -404,21 +448,29 @@ __device__ __forceinline__ void window_log_weights(const uint4 (&q)[kPipeMaxP], 
         }
 #pragma unroll
     for (int t = 0; t < kPipeMaxP; ++t)
-        lw[t] = (t < L && mnb[t] != -INFINITY) ? (far[t] ? mnb[t] - m[t] : 0.f) + (logf(snb[t]) - logf(sm[t]))
-                                              : -INFINITY;
+        lw[t] = (t < L && mnb[t] != -INFINITY)
+                    ? (mnb[t] - m[t] < -60.f ? mnb[t] - m[t] : 0.f) + (logf(snb[t]) - logf(sm[t]))
+                    : -INFINITY;
 }
 
-__global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolParams p, uint32_t slot_bytes)
+// NCH = ceil(dim / 256) hidden chunks per lane (dim <= 1024).  Every shared
+// memory offset is a compile-time constant from the lane's column of the
+// ring, every global one a constant from the lane's first chunk of a row.
+template <int NCH>
+__global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolParams p)
 {
+    constexpr uint32_t kFrame = (NCH + 1) * 512;   // one frame of a slot
+    constexpr uint32_t kSlot = kPipeMaxP * kFrame;
     extern __shared__ __align__(16) uint8_t pool_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // per warp: kPipe slots, then the slots' headers; slot_bytes and the
-    // header block are multiples of 16, so every cp.async destination is
-    // 16-byte aligned
-    uint8_t *ring = pool_smem + (size_t)warp * (kPipe * slot_bytes + kPipeHdr);
-    int2 *hdr = reinterpret_cast<int2 *>(ring + kPipe * slot_bytes);
-    const int n_chunks = p.dim >> 3, z_chunks = p.n_classes >> 3;
-    const uint32_t hid_bytes = (uint32_t)(p.P * p.dim * 2);   // a slot: P hidden rows, then P logit rows
+    uint8_t *ring = pool_smem + (size_t)warp * pipe_warp_bytes<NCH>();
+    int2 *hdr = reinterpret_cast<int2 *>(ring + kPipe * kSlot);
+    uint8_t *col = ring + 16 * lane;   // this lane's 16-byte column
+    const uint32_t col_s = smem_u32(col);
+    const int n_chunks = p.dim >> 3;
+    // bit i: this lane's chunk 32 i + lane exists
+    const uint32_t hl = n_chunks >= 32 * NCH ? (1u << NCH) - 1u : (1u << ((n_chunks - lane + 31) >> 5)) - 1u;
+    const bool zl = 8 * lane < p.n_classes;
     // windows gw, gw + stride, ...: at any moment the warps of the grid work
     // on neighbouring windows (DRAM pages shared), each keeping kPipe of its
     // own in flight
@@ -434,14 +486,18 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolP
     auto issue = [&](int s) {
         int f0 = 0, L = -1, seq;
         if (more && next < p.n_rows && w.find(next, lane, f0, L, seq)) {
-            uint8_t *slot = ring + (size_t)s * slot_bytes;
-            for (int t = 0; t < L; ++t) {
-                const __nv_bfloat16 *hrow = p.hidden + (long long)(f0 + t) * p.h_stride;
-                for (int ch = lane; ch < n_chunks; ch += 32)
-                    cp_async16(smem_u32(slot + (size_t)(t * p.dim + 8 * ch) * 2), hrow + 8 * ch);
-                if (lane < z_chunks)
-                    cp_async16(smem_u32(slot + hid_bytes + (size_t)(t * p.n_classes + 8 * lane) * 2),
-                               p.logits + (long long)(f0 + t) * p.z_stride + 8 * lane);
+            const uint32_t dst = col_s + s * kSlot;
+#pragma unroll
+            for (int t = 0; t < kPipeMaxP; ++t) {
+                if (t < L) {
+                    const __nv_bfloat16 *hrow = p.hidden + (long long)(f0 + t) * p.h_stride + 8 * lane;
+#pragma unroll
+                    for (int i = 0; i < NCH; ++i)
+                        if (hl >> i & 1u)
+                            cp_async16(dst + t * kFrame + i * 512, hrow + 256 * i);
+                    if (zl)
+                        cp_async16(dst + t * kFrame + NCH * 512, p.logits + (long long)(f0 + t) * p.z_stride + 8 * lane);
+                }
             }
         } else {
             more = false;
@@ -452,13 +508,11 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolP
         next += stride;
         cp_async_commit();
     };
-#pragma unroll
-    for (int s = 0; s < kPipe - 1; ++s)
-        issue(s);
+    issue(0);
     long long last = -1;   // the last window this warp pooled
-    for (long long g = gw, k = 0; g < p.n_rows; g += stride, ++k) {
-        const int s = (int)(k % kPipe);
-        issue((s + kPipe - 1) % kPipe);   // this warp's window k + kPipe - 1, into the slot freed last pass
+    int s = 0;
+    for (long long g = gw; g < p.n_rows; g += stride, s ^= 1) {
+        issue(s ^ 1);                     // this warp's next window, into the slot freed last pass
         cp_async_wait<kPipe - 1>();       // this lane's copies of window g have landed
         __syncwarp();
         const int2 hd = hdr[s];
@@ -466,13 +520,13 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolP
             break;   // past the batch's last window
         const int f0 = hd.x, L = hd.y;
         last = g;
-        const uint8_t *slot = ring + (size_t)s * slot_bytes;
+        const uint8_t *src = col + s * kSlot;
         uint4 zq[kPipeMaxP];
 #pragma unroll
         for (int t = 0; t < kPipeMaxP; ++t) {
             zq[t] = make_uint4(0u, 0u, 0u, 0u);
-            if (t < L && lane < z_chunks)
-                zq[t] = *reinterpret_cast<const uint4 *>(slot + hid_bytes + (size_t)(t * p.n_classes + 8 * lane) * 2);
+            if (t < L && zl)
+                zq[t] = *reinterpret_cast<const uint4 *>(src + t * kFrame + NCH * 512);
         }
         float lw[kPipeMaxP];
         window_log_weights(zq, p.n_classes, L, lane, lw);
@@ -492,26 +546,32 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolP
             r[t] = (t < L && M != -INFINITY) ? exp2f((lw[t] - M) * kLog2e) : 0.f;   // 0 for a weight of 0
             wsum += r[t];
         }
-        const float inv = M != -INFINITY ? 1.f / wsum : 0.f;   // wsum >= 1 when some weight is not 0
-        __nv_bfloat16 *orow = p.pooled + g * (long long)p.dim;
-        for (int ch = lane; ch < n_chunks; ch += 32) {
-            uint4 res = make_uint4(0u, 0u, 0u, 0u);
-            if (M != -INFINITY) {
-                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // wsum >= 1 when some weight is not 0; the frames' weights are
+        // normalised before the FMAs
+        const float inv = M != -INFINITY ? 1.f / wsum : 0.f;
 #pragma unroll
-                for (int t = 0; t < kPipeMaxP; ++t) {
-                    if (t < L) {
-                        float v[8];
-                        chunk_vals(*reinterpret_cast<const uint4 *>(slot + (size_t)(t * p.dim + 8 * ch) * 2), v);
+        for (int t = 0; t < kPipeMaxP; ++t)
+            r[t] *= inv;
+        __nv_bfloat16 *orow = p.pooled + g * (long long)p.dim + 8 * lane;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            acc[e] = fmaf(r[t], v[e], acc[e]);
-                    }
+        for (int i = 0; i < NCH; ++i) {
+            if (!(hl >> i & 1u))
+                continue;
+            float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+            for (int t = 0; t < kPipeMaxP; ++t) {
+                if (t < L && M != -INFINITY) {   // every weight 0: a zero row, whatever the frames hold
+                    float v[8];
+                    chunk_vals(*reinterpret_cast<const uint4 *>(src + t * kFrame + i * 512), v);
+                    const float2 rr = make_float2(r[t], r[t]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        acc[e] = ffma2(make_float2(v[2 * e], v[2 * e + 1]), rr, acc[e]);
                 }
-                res = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                                 pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
             }
-            __stcs(reinterpret_cast<uint4 *>(orow + 8 * ch), res);
+            const uint4 res = make_uint4(pack_bf16x2(acc[0].x, acc[0].y), pack_bf16x2(acc[1].x, acc[1].y),
+                                         pack_bf16x2(acc[2].x, acc[2].y), pack_bf16x2(acc[3].x, acc[3].y));
+            __stcs(reinterpret_cast<uint4 *>(orow + 256 * i), res);
         }
         __syncwarp();   // slot s is refilled by the next pass
     }
@@ -526,6 +586,24 @@ __global__ void __launch_bounds__(kPoolThreads) posterior_pool_pipe_kernel(PoolP
     }
     if (w.bad && lane == 0)
         report(p.status, NLE_ERR_INVALID_ARG);
+}
+
+template <int NCH>
+int launch_pool_pipe(const PoolParams &p, const nle::DeviceInfo &di, int dev, cudaStream_t stream)
+{
+    constexpr size_t smem_cta = (size_t)kPoolWarps * pipe_warp_bytes<NCH>();
+    int per_sm = (int)((size_t)di.smem_optin / (smem_cta + 1024));
+    per_sm = per_sm < 1 ? 1 : (per_sm > 6 ? 6 : per_sm);
+    long long warps = (long long)di.sm_count * per_sm * kPoolWarps;
+    if (warps > p.n_rows)
+        warps = p.n_rows;
+    const long long ctas = (warps + kPoolWarps - 1) / kPoolWarps;
+    if (smem_cta > 48 * 1024 &&
+        !nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(posterior_pool_pipe_kernel<NCH>), dev,
+                                     di.smem_optin))
+        return NLE_ERR_CUDA;
+    posterior_pool_pipe_kernel<NCH><<<(int)ctas, kPoolThreads, smem_cta, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
 }
 
 } // namespace
@@ -574,20 +652,13 @@ extern "C" int nle_posterior_pool_fwd(const void *hidden, int64_t hidden_stride,
     const int grid = (int)(ctas < cap ? ctas : cap);
     const bool vec = (reinterpret_cast<uintptr_t>(logits) & 15) == 0 && logits_stride % 8 == 0 && n_classes % 8 == 0;
     if (vec && n_classes <= 256 && dim <= 1024 && pool_frames <= kPipeMaxP) {
-        const uint32_t slot = (uint32_t)(pool_frames * (dim + n_classes) * 2);
-        const size_t smem_cta = (size_t)kPoolWarps * (kPipe * slot + kPipeHdr);
-        int per_sm = (int)((size_t)di.smem_optin / (smem_cta + 1024));
-        per_sm = per_sm < 1 ? 1 : (per_sm > 6 ? 6 : per_sm);
-        long long warps = (long long)di.sm_count * per_sm * kPoolWarps;
-        if (warps > n_pooled_rows)
-            warps = n_pooled_rows;
-        const long long ctas = (warps + kPoolWarps - 1) / kPoolWarps;
-        if (smem_cta > 48 * 1024 && !nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(posterior_pool_pipe_kernel),
-                                                                 dev, di.smem_optin))
-            return NLE_ERR_CUDA;
-        posterior_pool_pipe_kernel<<<(int)ctas, kPoolThreads, smem_cta, static_cast<cudaStream_t>(stream)>>>(
-            p, slot);
-        return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
+        const cudaStream_t st = static_cast<cudaStream_t>(stream);
+        switch ((dim / 8 + 31) / 32) {
+        case 1: return launch_pool_pipe<1>(p, di, dev, st);
+        case 2: return launch_pool_pipe<2>(p, di, dev, st);
+        case 3: return launch_pool_pipe<3>(p, di, dev, st);
+        default: return launch_pool_pipe<4>(p, di, dev, st);
+        }
     }
     // per-warp log weights of a window: above 48 KB (pool_frames > 3072)
     // the kernel needs the opt-in shared memory limit

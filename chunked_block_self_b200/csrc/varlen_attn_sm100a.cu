@@ -76,6 +76,14 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 128;                         // per chain: S (64 columns), then O
 constexpr uint32_t kOCol = 64;
 constexpr int kSeg = 32;                                    // softmax register segment (2 per key tile)
+constexpr int kDescRing = 4;                                // item descriptors in flight
+constexpr int kDescReaders = 4 * kChains;                   // every chain warp reads every descriptor
+
+// One work item as the producer publishes it to the chain warps (L < 0:
+// no further item).
+struct ItemDesc {
+    int f0, L, T, h;
+};
 
 struct Bars {
     uint64_t q_full[2];
@@ -87,6 +95,9 @@ struct Bars {
     uint64_t wg_p[kChains];      // 4 arrivals: P of the tile written
     uint64_t o_done[kChains];    // the chain's latest PV MMA has completed
     uint64_t mma_done[kChains];
+    uint64_t desc_full[kDescRing];
+    uint64_t desc_empty[kDescRing];   // kDescReaders arrivals: every chain warp has read the entry
+    ItemDesc desc[kDescRing];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -153,20 +164,53 @@ __device__ __forceinline__ void tma_load_2d_nohint(uint32_t dst, const void *tma
                  : "memory");
 }
 
+// p = exp2(s * sl2 - m) for the W keys of a segment (masked keys hold -inf
+// -> 0), packed to bf16 pairs and stored over S's columns [C0/2, C0/2 +
+// W/2) eight at a time: the S values they overwrite are already in
+// registers.  Two partial sums and maxima and eight packed registers at a
+// time keep the chain warps within their 96 registers.  Returns the
+// segment sum; ymax: the largest exponent.
+template <int W>
+__device__ __forceinline__ float seg_exp_store(uint32_t tP, const uint32_t (&s)[kSeg], float sl2, float m,
+                                               float &ymax)
+{
+    static_assert(W % 16 == 0 && W <= kSeg, "segment width");
+    float ls[2] = {0.f, 0.f};
+    float ym[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < W / 2; c += 8) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = 2 * (c + j);
+            const float ya = fmaf(__uint_as_float(s[i]), sl2, -m);
+            const float yb = fmaf(__uint_as_float(s[i + 1]), sl2, -m);
+            ym[j & 1] = fmax3(ym[j & 1], ya, yb);
+            const float pa = ex2_approx(ya);
+            const float pb = ex2_approx(yb);
+            ls[j & 1] += pa + pb;
+            pk[j] = pack_bf16x2(pa, pb);
+        }
+        tmem_st8p(tP + c, pk);
+    }
+    ymax = fmaxf(ym[0], ym[1]);
+    return ls[0] + ls[1];
+}
+
 // One segment of a key tile (whole warp): p for its W keys from the S values
 // in `cur` (keys past the tile's valid ones already -inf), with the rare
 // shift step of the block kernel's softmax, but done from registers: for a
 // row whose exponent went past kYMax, the segment's exact max gives k, m
 // moves up by k, the running sum and the product fs of this tile's factors
-// take 2^-k, the segment is recomputed and the P already written in this
-// tile (columns < C0/2) are rescaled (other rows: k = 0, unchanged).
+// take 2^-k, the segment is recomputed (its P stored again over the first
+// attempt's) and the P already written in this tile (columns < C0/2) are
+// rescaled (other rows: k = 0, unchanged).
 template <int W>
 __device__ __forceinline__ void tile_segment(uint32_t tS, int C0, uint32_t (&cur)[kSeg], float sl2, float &m,
                                              float &l, float &fs)
 {
-    uint32_t pk[W / 2];
     float ymax;
-    float ls = seg_exp<W>(cur, pk, sl2, m, ymax);
+    float ls = seg_exp_store<W>(tS + C0 / 2, cur, sl2, m, ymax);
     const bool mine = !(ymax <= kYMax);   // this row's exponent is too large (or NaN)
     if (__any_sync(kFull, mine)) {
         // only the rows that need it move their shift, so a row's result
@@ -177,12 +221,12 @@ __device__ __forceinline__ void tile_segment(uint32_t tS, int C0, uint32_t (&cur
         m += (float)k;
         l *= f;
         fs *= f;
-        ls = seg_exp<W>(cur, pk, sl2, m, ymax);
+        tmem_wait_st();   // the first attempt's stores complete before they are overwritten
+        ls = seg_exp_store<W>(tS + C0 / 2, cur, sl2, m, ymax);
         if (C0 > 0)
             rescale_p(tS, C0 / 2, f);
     }
     l += ls;
-    seg_store<W>(tS + C0 / 2, pk);
 }
 
 // Softmax of one key tile for this lane's row: keys [0, nv) of the tile are
@@ -266,6 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&bars->o_done[c]), 1);
             mbar_init(smem_u32(&bars->mma_done[c]), 1);
         }
+        for (int j = 0; j < kDescRing; ++j) {
+            mbar_init(smem_u32(&bars->desc_full[j]), 1);
+            mbar_init(smem_u32(&bars->desc_empty[j]), kDescReaders);
+        }
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -291,13 +339,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         it.init(p, lane);
         const uint64_t pol_q = policy_evict_first();   // Q is read once; K and V by every query unit
         const bool skip0 = (p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) != 0;
-        int nq = 0;    // items whose Q stage was claimed
+        int nq = 0;    // items whose Q stage was claimed (= descriptors published)
         int nkt = 0;   // key tiles whose KV stage was claimed
         bool stop = false;
+        // the chain warps learn each item (and the end) from the descriptor
+        // ring, so they hold no plan-walking state
+        auto publish = [&](const ItemDesc &d) -> bool {
+            const int j = nq % kDescRing;
+            if (nq >= kDescRing && !wait_bar(smem_u32(&bars->desc_empty[j]), (uint32_t)(nq / kDescRing - 1) & 1,
+                                             abort_flag, wait_ns, p.status))
+                return false;
+            if (lane == 0) {
+                bars->desc[j] = d;
+                mbar_arrive(smem_u32(&bars->desc_full[j]));
+            }
+            __syncwarp();
+            return true;
+        };
         for (;;) {
             int f0, L, us, T, h;
             if (!it.next(p, lane, f0, L, us, T, h))
                 break;
+            if (!publish(ItemDesc{f0, L, T, h})) {
+                stop = true;
+                break;
+            }
             const int qs = nq & 1;
             if (nq >= 2 && !wait_bar(smem_u32(&bars->q_empty[qs]), (uint32_t)((nq >> 1) - 1) & 1, abort_flag,
                                      wait_ns, p.status))
@@ -335,6 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (it.w.bad && lane == 0)
             report(p.status, NLE_ERR_INVALID_ARG);
+        if (!stop)
+            publish(ItemDesc{0, -1, 0, 0});   // end marker (its index is nq, not counted as an item)
         // drain: the last copy into each stage must land before exit
         if (lane == 0) {
             for (int m = nq - 2; m < nq; ++m)
@@ -387,16 +455,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tS = slot + ((uint32_t)(qq * 32) << 16);
         const float sl2 = p.scale_log2;
         const uint32_t id_pv = idesc_bf16_f32(128, 64, true);
-        ItemWalk it;
-        it.init(p, lane);
         int n = 0;           // items
         int nkt = 0;         // key tiles walked (KV stage sequence)
         uint32_t uses = 0;   // S/PV rounds of this chain
         bool ok = true;
         for (;; ++n) {
-            int f0, L, us, T, h;
-            if (!it.next(p, lane, f0, L, us, T, h))
+            const int dj = n % kDescRing;
+            if (!wait_bar(smem_u32(&bars->desc_full[dj]), (uint32_t)(n / kDescRing) & 1, abort_flag, wait_ns,
+                          p.status)) {
+                ok = false;
                 break;
+            }
+            // the entry stays claimed until the item's output is written:
+            // its first frame and head are read again there
+            const int L = bars->desc[dj].L, T = bars->desc[dj].T;
+            if (L < 0) {
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_u32(&bars->desc_empty[dj]));
+                break;   // no further item
+            }
             const int qs = n & 1;
             const int tiles = (T + kKeys - 1) / kKeys;
             const bool chain_rows = L > c * kQRows;
@@ -410,6 +488,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!chain_rows) {
                 // no query rows for this chain: release the item's Q and KV
                 // stages in order (each only once it holds this item's data)
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_u32(&bars->desc_empty[dj]));
                 if (leader) {
                     if (lane == 0)
                         mbar_arrive(smem_u32(&bars->q_empty[qs]));
@@ -516,6 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // O in two halves of 32 columns (registers are scarce at 20 warps)
                 const float inv = 1.f / l;
                 const bool row_ok = row0 + lane < L;
+                const int f0 = bars->desc[dj].f0, h = bars->desc[dj].h;
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + (size_t)(f0 + row0 + lane) * p.out_stride + h * 64);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -538,6 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bars->desc_empty[dj]));
         }
         // this chain's MMAs must finish before TMEM is released
         if (leader) {

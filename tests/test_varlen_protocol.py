@@ -6,7 +6,10 @@ producer warp (each item's Q into one of two Q stages, then the utterance's
 to the chains once it has landed, and four chains of four warps.  Every
 chain walks every K/V tile of every item (a stage is freed by four
 arrivals); a chain without query rows in an item only waits for each stage
-to hold the item's data and releases it.  Per tile a chain's first warp
+to hold the item's data and releases it.  The chains learn each item, and
+the end, from a ring of item descriptors that the producer fills (an entry
+is freed by all sixteen chain warps: at once by a warp without rows in the
+item, after the item's output otherwise).  Per tile a chain's first warp
 waits for the stage and for its previous PV MMA, issues S, the chain's four
 warps wait for S and write P, and the first warp issues PV.
 
@@ -36,7 +39,7 @@ class _Bar:
             self.pending, self.phases = 0, self.phases + 1
 
 
-def _simulate(items, nkv, seed, p_complete=0.3, p_out_of_order=0.2, early_release=False):
+def _simulate(items, nkv, seed, p_complete=0.3, p_out_of_order=0.2, early_release=False, ndesc=4):
     """items: (query rows L, utterance length T) of the CTA's items in order."""
     rnd = random.Random(seed)
     bars = {}
@@ -50,14 +53,23 @@ def _simulate(items, nkv, seed, p_complete=0.3, p_out_of_order=0.2, early_releas
         bar(f"kv_full{s}"), bar(f"kv_ready{s}"), bar(f"kv_empty{s}", CHAINS)
     for c in range(CHAINS):
         bar(f"s_full{c}"), bar(f"wg_p{c}", 4), bar(f"o_done{c}")
+    for j in range(ndesc):
+        bar(f"desc_full{j}"), bar(f"desc_empty{j}", 4 * CHAINS)
     later = []   # async completions (TMA copies, MMA commits)
 
     def tiles(T):
         return (T + KEYS - 1) // KEYS
 
+    def publish(n):
+        j = n % ndesc
+        if n >= ndesc:
+            yield f"desc_empty{j}", n // ndesc - 1
+        bars[f"desc_full{j}"].arrive()
+
     def producer():
         nkt = 0
         for nq, (L, T) in enumerate(items):
+            yield from publish(nq)
             qs = nq & 1
             if nq >= 2:
                 yield f"q_empty{qs}", (nq >> 1) - 1
@@ -68,6 +80,7 @@ def _simulate(items, nkv, seed, p_complete=0.3, p_out_of_order=0.2, early_releas
                     yield f"kv_empty{s}", u - 1
                 later.append(f"kv_full{s}")
                 nkt += 1
+        yield from publish(len(items))   # end marker
 
     def fixup():
         nkt = 0
@@ -82,10 +95,13 @@ def _simulate(items, nkv, seed, p_complete=0.3, p_out_of_order=0.2, early_releas
         nkt, uses = 0, 0
         for n, (L, T) in enumerate(items):
             qs, nt = n & 1, tiles(T)
+            dj = n % ndesc
+            yield f"desc_full{dj}", n // ndesc
             if leader:
                 yield f"q_full{qs}", n >> 1
             if L <= c * QROWS:
                 # no rows of this chain: release the item's stages in order
+                bars[f"desc_empty{dj}"].arrive()
                 if leader:
                     bars[f"q_empty{qs}"].arrive()
                     for j in range(nt):
@@ -113,6 +129,10 @@ def _simulate(items, nkv, seed, p_complete=0.3, p_out_of_order=0.2, early_releas
                 uses += 1
                 nkt += 1
             yield f"o_done{c}", uses - 1
+            bars[f"desc_empty{dj}"].arrive()   # the output step read the entry again
+        n = len(items)
+        yield f"desc_full{n % ndesc}", n // ndesc   # the end marker
+        bars[f"desc_empty{n % ndesc}"].arrive()
 
     roles = {"producer": producer(), "fixup": fixup()}
     for c in range(CHAINS):
@@ -163,6 +183,17 @@ def test_varlen_kernel_barrier_phases(nkv):
         items = _items(rng, rng.randint(1, 7))
         _simulate(items, nkv, trial)
         _simulate(items, nkv, trial, p_complete=0.05, p_out_of_order=1.0)
+
+
+@pytest.mark.parametrize("ndesc", [1, 2, 3])
+def test_shallow_descriptor_rings(ndesc):
+    """The protocol holds for any ring depth (the kernel uses 4), up to one
+    entry: the producer then waits for every chain warp's output step."""
+    rng = random.Random(100 + ndesc)
+    for trial in range(60):
+        items = _items(rng, rng.randint(1, 7))
+        _simulate(items, 3, trial, ndesc=ndesc)
+        _simulate(items, 2, trial, p_complete=0.05, p_out_of_order=1.0, ndesc=ndesc)
 
 
 def test_model_catches_an_early_stage_release():

@@ -64,9 +64,9 @@ NCU_TRAFFIC = {
                     "traffic_over_algorithmic": (265965568 + 7668992) / 290320384},
     # full-utterance attention: the long-clip workload, the same launch as the bench's
     "varlen_attn": {"files": ('varlen_attn_sm100a.cu', 'attn_softmax.cuh', 'nle_device.cuh'),
-                   "source_sha256": "9f9034f668362301b35d9d87571d4a0718ac495d5026e1ceed7ccc202e3f0714",
-                   "traffic_over_algorithmic": (343928832 + 91376128) / 439304192,
-                   "tensor_pipe_pct": 25.5},
+                   "source_sha256": "f687eb567c9643601dca019254550645b968652fd7c4f8d2a9e54cf02edc976e",
+                   "traffic_over_algorithmic": (345912064 + 88160512) / 439304192,
+                   "tensor_pipe_pct": 27.2},
     # fused projection + block attention on the batch-128 workload (d_model 1024,
     # 16 heads); DRAM writes sit below the output's bytes because part of it is
     # still in L2 when the kernel ends
@@ -76,8 +76,8 @@ NCU_TRAFFIC = {
                  "tensor_pipe_pct": 44.4},
     # posterior pooling over the whole batch-128 workload (58,903 frames)
     "posterior_pool": {"files": ('pool_sm100a.cu', 'nle_device.cuh'),
-                       "source_sha256": "b8d5d604258c92eaf69cbb051ec3912c14a782103b9afa75ecac9a378f4211db",
-                       "traffic_over_algorithmic": (151211776 + 28471552) / 211398236},
+                      "source_sha256": "377b218edef5a26471eb2a6eb04fe40a21a24780c34f4a3b9fcb1405a51f5f2a",
+                      "traffic_over_algorithmic": (150827776 + 28794368) / 211398236},
     # CTC argmax: captured on 16 utterances (3,300 rows, 662.4 MB); traffic grows
     # with rows, so the ratio is applied to the full batch
     "ctc_argmax": {"files": ('ctc_sm100a.cu', 'nle_device.cuh'),
@@ -345,15 +345,21 @@ def run_reference(args, rank, world):
     return 0
 
 
-def time_launches(fn, stream, reps, flush=None):
+def time_launches(fn, stream, reps, flush=None, clean=False):
     """Median and mean (ms) of `reps` launches of fn, each bracketed by CUDA
-    events on `stream`; with `flush`, a write of that buffer (larger than
-    L2) precedes every launch (and keeps the GPU busy while the launch is
-    queued, so the first event is taken right before the kernel starts)."""
+    events on `stream` (torch's current stream); with `flush`, a write of
+    that buffer (larger than L2) precedes every launch (and keeps the GPU
+    busy while the launch is queued, so the first event is taken right
+    before the kernel starts).  The write leaves L2 full of dirty lines,
+    which the timed launch then writes back as it evicts them; with
+    `clean`, the buffer is also read back before the launch, so L2 holds
+    only clean lines of it (still none of the kernel's inputs)."""
     ts = []
     for _ in range(reps):
         if flush is not None:
             flush.fill_(1)
+            if clean:
+                flush.view(torch.int64).sum()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
@@ -640,13 +646,18 @@ def run_nle(args, rank, world, local):
         for _ in range(3):
             pool_step()
         pool_ms = timed(pool_step, 50)
+        pool_clean_ms = time_launches(pool_step, stream, 50, flush, clean=True)[0]
         # hidden and logits once, pooled rows and weights written
         pool_bytes = n_fr * (wl.HIDDEN_DIM + wl.CHAR_CLASSES) * 2 + n_rows * wl.HIDDEN_DIM * 2 + n_fr * 4
         pool = {"frames": n_fr, "rows": n_rows, "pool_frames": wl.POOL_FRAMES, "dim": wl.HIDDEN_DIM,
                 "char_classes": wl.CHAR_CLASSES, "ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
                 "algorithmic_bytes": pool_bytes, "traffic": ncu_traffic("posterior_pool", pool_bytes),
                 "l2": "flushed (256 MB write) before each launch", "kernels": 1,
-                "timing": "median of 50 launches"}
+                "timing": "median of 50 launches",
+                # the same launches after the flush is also read back: the
+                # flush's dirty lines are written out before the launch
+                # instead of during it
+                "ms_clean_l2": pool_clean_ms, "gbs_clean_l2": pool_bytes / (pool_clean_ms * 1e-3) / 1e9}
         del px, pooled, pw
 
         logits = wl.ctc_logits(rows_u, seed=wl.default_seed(CFG) + 3000 + rank, device=dev)
@@ -725,6 +736,8 @@ def run_nle(args, rank, world, local):
     for extra in (pool, ctc):
         if extra is not None:
             extra["pct_of_hbm_peak"] = 100.0 * extra["gbs"] / hbm_peak
+    if pool is not None:
+        pool["pct_of_hbm_peak_clean_l2"] = 100.0 * pool["gbs_clean_l2"] / hbm_peak
     achieved_gbs = by_blk / (t_blk * 1e-3) / 1e9
     traffic = ncu_traffic("block_attn", by_blk)
     blk_tflops = f_blk / (t_blk * 1e-3) / 1e12

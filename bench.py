@@ -14,7 +14,7 @@ HBM before timing; each kernel is also timed alone (median over the K
 steps).  One JSON line is printed by rank 0.
 
 The `configs` field of the line times the kernels on all five workloads
-(median of >= 50 launches each, L2 flushed by a 256 MB write before every
+(median of >= 50 launches each, L2 flushed by a write of twice the L2 size before every
 launch, and back to back for the two small workloads that fit in L2).
 
 Multi-GPU (torchrun, one process per GPU): data-parallel replicas, each
@@ -345,6 +345,13 @@ def run_reference(args, rank, world):
     return 0
 
 
+def l2_flush_buffer(dev):
+    """A buffer twice the device's L2 (its size read at run time): writing it
+    before a launch evicts everything the previous launch left in L2."""
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or (126 << 20))
+    return torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+
 def time_launches(fn, stream, reps, flush=None, clean=False):
     """Median and mean (ms) of `reps` launches of fn, each bracketed by CUDA
     events on `stream` (torch's current stream); with `flush`, a write of
@@ -394,7 +401,7 @@ def measure_configs(nle, dev, stream, reps, rank, hbm_peak, tf_peak):
     two small workloads (which fit in L2) are also timed hot: `reps`
     launches queued back to back, mean per launch (median of 5 runs)."""
     sp = stream.cuda_stream
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = l2_flush_buffer(dev)
     res = {}
     for c in (1, 2, 3, 4, 5):
         seed = wl.default_seed(c) + rank
@@ -474,7 +481,7 @@ def measure_qkv_attn(nle, dev, stream, reps, rank, lengths, tf_peak):
     w = wl.device_normal((3 * heads * 64, dm), 1.0 / 32.0, seed + 1, dev)
     b = wl.device_normal((3 * heads * 64,), 0.5, seed + 2, dev)
     out = torch.empty((T, heads, 64), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = l2_flush_buffer(dev)
 
     def fused():
         nle.nle_block_attn_qkv_fwd(x, w, b, out, cu, block_frames=B, stream=sp)
@@ -500,7 +507,8 @@ def measure_qkv_attn(nle, dev, stream, reps, rank, lengths, tf_peak):
     byt = 2 * (T * dm + 3 * heads * 64 * dm + 3 * heads * 64 + T * heads * 64)   # X, W, b read; O written
     res = {"workload": f"config {CFG} utterances ({len(lengths)}, {T} frames), d_model {dm}, {heads} heads x 64, "
                        "synthetic X ~ N(0,1), W ~ N(0,1/1024), bias ~ N(0,0.25), bf16",
-           "ms": med, "ms_mean": mean, "timing": f"median of {reps} launches, L2 flushed (256 MB write) before each",
+           "ms": med, "ms_mean": mean,
+           "timing": f"median of {reps} launches, L2 flushed (a write of twice the L2 size) before each",
            "algorithmic_flops": flops, "projection_flops": f_proj, "attention_flops": f_att,
            "tflops": tflops, "pct_of_dense_bf16_peak": 100.0 * tflops / tf_peak,
            "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_peak, "unit": "TFLOP/s",
@@ -631,7 +639,7 @@ def run_nle(args, rank, world, local):
         rows_u = [-(-int(t) // wl.POOL_FRAMES) for t in clen]
         cu_r = torch.from_numpy(wl.cu_seqlens(rows_u)).to(dev)
         n_rows, n_fr = int(sum(rows_u)), int(sum(int(t) for t in clen))
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        flush = l2_flush_buffer(dev)
 
         def timed(fn, reps):
             return time_launches(fn, stream, reps, flush)[0]   # median
@@ -652,7 +660,7 @@ def run_nle(args, rank, world, local):
         pool = {"frames": n_fr, "rows": n_rows, "pool_frames": wl.POOL_FRAMES, "dim": wl.HIDDEN_DIM,
                 "char_classes": wl.CHAR_CLASSES, "ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
                 "algorithmic_bytes": pool_bytes, "traffic": ncu_traffic("posterior_pool", pool_bytes),
-                "l2": "flushed (256 MB write) before each launch", "kernels": 1,
+                "l2": "flushed (a write of twice the L2 size) before each launch", "kernels": 1,
                 "timing": "median of 50 launches",
                 # the same launches after the flush is also read back: the
                 # flush's dirty lines are written out before the launch
@@ -676,7 +684,7 @@ def run_nle(args, rank, world, local):
         ctc_bytes = logits.numel() * 2 + n_rows * 12 + len(clen) * 4
         ctc = {"rows": n_rows, "utterances": len(clen), "classes": int(logits.shape[1]), "ms": ctc_ms,
                "rows_per_s": n_rows / (ctc_ms * 1e-3), "gbs": ctc_bytes / (ctc_ms * 1e-3) / 1e9,
-               "algorithmic_bytes": ctc_bytes, "l2": "flushed (256 MB write) before each launch", "kernels": 2,
+               "algorithmic_bytes": ctc_bytes, "l2": "flushed (a write of twice the L2 size) before each launch", "kernels": 2,
                "timing": "median of 20 launches",
                # the argmax kernel's DRAM bytes (logits once, classes written)
                "traffic_argmax": ncu_traffic("ctc_argmax", logits.numel() * 2 + n_rows * 4)}

@@ -79,9 +79,11 @@ def test_golden_cases(case, cuda_device):
 @pytest.mark.parametrize("P,dim,n_classes,pads", [
     (2, 1024, 256, (0, 0)), (1, 8, 1, (0, 0)), (2, 8, 2, (8, 1)), (3, 24, 37, (16, 3)), (4, 1024, 256, (8, 5)),
     (7, 64, 1000, (0, 7)), (2, 1032, 2, (0, 0)), (16, 128, 5, (0, 2)),
-    # the pipelined path (P <= 4, dim <= 1024, classes <= 256 in 16-byte chunks)
+    # the pipelined path (P <= 2, dim <= 1024, classes <= 256 in 16-byte chunks), with 1-4
+    # hidden chunks per lane, some lanes without a chunk, and fewer than 32 logit chunks
     (1, 1024, 256, (0, 0)), (3, 64, 8, (8, 8)), (4, 1024, 256, (8, 0)), (2, 8, 16, (0, 0)),
-    (4, 1000, 248, (16, 8))])
+    (4, 1000, 248, (16, 8)), (2, 512, 64, (0, 0)), (2, 640, 128, (8, 8)), (1, 264, 8, (0, 0)),
+    (2, 776, 200, (24, 16)), (2, 1000, 256, (0, 0))])
 def test_random_shapes(P, dim, n_classes, pads, cuda_device):
     lengths = [37, 0, 1, 200, 5, 64, 3]
     cu = wl.cu_seqlens(lengths)

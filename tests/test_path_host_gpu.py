@@ -84,3 +84,33 @@ def test_host_path_rejects_bad_tables():
     assert call(b2, QW * n_win) == nle.NLE_ERR_INVALID_ARG
     b3 = nle.PathBuffers(*([dummy] * 8), cu.ctypes.data, *([dummy] * 8), None)   # no device cu
     assert call(b3, QW * n_win) == nle.NLE_ERR_INVALID_ARG
+
+
+@pytest.mark.gpu
+def test_host_path_full_batch_against_oracle(cuda_device):
+    """The whole batch-128 workload (128 utterances, 58,903 frames, 3,992
+    windows) through the host-memory entry point with its default chunking:
+    bit-equal to the device path, and every output of both kernels within
+    the path's tolerance of the fp64 oracle (rel-L2 <= 5e-3, max-abs <= 2e-2
+    per tensor)."""
+    import oracle
+
+    host = {n: t.pin_memory() for n, t in _inputs(128, seed=503).items()}
+    ref, ref_w = _device_reference(host, cuda_device)
+    dev = {n: torch.empty(t.shape, dtype=t.dtype, device=cuda_device) for n, t in host.items()}
+    host["out"].fill_(float("nan"))
+    host["out_w"].fill_(float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    nle.nle_path_fwd_host(host, dev, block_frames=B, window_frames=W, queries_per_window=QW, dev_status=status)
+    torch.cuda.current_stream().synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(host["out"], ref)
+    assert torch.equal(host["out_w"], ref_w)
+    cu = host["cu"].numpy()
+    want = oracle.block_attn(host["q"], host["k"], host["v"], cu, block_frames=B)
+    want_w = oracle.window_xattn(host["qw"], host["kw"], host["vw"], cu, window_frames=W, queries_per_window=QW)
+    for got, exp in ((host["out"], want), (host["out_w"], want_w)):
+        g = got.float().numpy().astype(np.float64)
+        err = g - exp
+        rel = np.linalg.norm(err) / np.linalg.norm(exp)
+        assert rel <= 5e-3 and np.abs(err).max() <= 2e-2, f"rel_l2={rel:.3e} max_abs={np.abs(err).max():.3e}"

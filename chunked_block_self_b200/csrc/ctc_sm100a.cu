@@ -33,6 +33,8 @@ namespace {
 using namespace nle;
 
 constexpr int kArgmaxThreads = 256;
+constexpr int kArgmaxCtasPerSm = 4;   // 55 registers: four CTAs of 256 threads fit an SM
+constexpr int kArgmaxUnroll = 8;      // 16-byte loads in flight per thread (32 KB per CTA)
 constexpr int kCollapseThreads = 256;
 
 // (value, class) pair order: larger value first, then the lower class.
@@ -67,14 +69,15 @@ __device__ __forceinline__ float chunk_elem(const uint4 &q, int e)
     return e & 1 ? bf16_hi(w) : bf16_lo(w);
 }
 
-// Per frame: a CTA reads the row's whole 16-byte chunks with 16-byte loads
-// and keeps, per thread, only the largest chunk maximum, the first chunk
-// that reached it and that chunk's 8 values (packed bf16 max: about one
-// instruction per logit, so the loop stays under the HBM time); the class
-// inside that chunk is found from the kept values, so no logit is read
-// twice.  The row's elements before its first 16-byte boundary and after its
+// Per frame: a CTA reads the row's whole 16-byte chunks with 16-byte loads,
+// eight in flight per thread (128 KB per SM: enough to cover DRAM latency at
+// full bandwidth), and keeps, per thread, only the largest chunk maximum,
+// the first chunk that reached it and that chunk's 8 values (packed bf16 max:
+// about one instruction per logit, so the loop stays under the HBM time);
+// the class inside that chunk is found from the kept values, so no logit is
+// read twice.  The row's elements before its first 16-byte boundary and after its
 // last one (at most 7 each) are read one by one.
-__global__ void __launch_bounds__(kArgmaxThreads)
+__global__ void __launch_bounds__(kArgmaxThreads, kArgmaxCtasPerSm)
     ctc_argmax_kernel(const __nv_bfloat16 *__restrict__ logits, long long row_stride, int n_classes,
                       long long total_frames, int32_t *__restrict__ frame_class)
 {
@@ -94,13 +97,13 @@ __global__ void __launch_bounds__(kArgmaxThreads)
         int bk = -1;   // first chunk of this thread whose maximum is best (-1: none above -inf)
         uint4 bq = make_uint4(0u, 0u, 0u, 0u);   // that chunk's values
         int k = tid;
-        for (; k + 3 * kArgmaxThreads < nfull; k += 4 * kArgmaxThreads) {
-            uint4 q[4];
+        for (; k + (kArgmaxUnroll - 1) * kArgmaxThreads < nfull; k += kArgmaxUnroll * kArgmaxThreads) {
+            uint4 q[kArgmaxUnroll];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < kArgmaxUnroll; ++j)
                 q[j] = __ldcs(chunks + k + j * kArgmaxThreads);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < kArgmaxUnroll; ++j) {
                 const float f = chunk_max(q[j]);
                 if (f > best) {
                     best = f;
@@ -255,7 +258,9 @@ extern "C" int nle_ctc_greedy_fwd(const void *logits, int64_t row_stride, int n_
         return NLE_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (total_frames > 0) {
-        const long long grid = total_frames < (long long)di.sm_count * 8 ? total_frames : (long long)di.sm_count * 8;
+        // every CTA resident at once; rows in a grid-stride loop
+        const long long cap = (long long)di.sm_count * kArgmaxCtasPerSm;
+        const long long grid = total_frames < cap ? total_frames : cap;
         ctc_argmax_kernel<<<(int)grid, kArgmaxThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(logits),
                                                                  (long long)row_stride, n_classes, total_frames,
                                                                  frame_class);

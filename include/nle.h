@@ -200,7 +200,7 @@ int nle_window_xattn_fwd_ex(const void *q, const void *k, const void *v,
  * Installation": packed sequences, is_causal=False): for every utterance i
  * and head h,  O = softmax(scale * Q K^T) V  over all T_i frames of the
  * utterance -- block attention with one block per utterance.  Keys are
- * walked in tiles of 128 with an online softmax (fp32, exact power-of-two
+ * walked in tiles of 64 with an online softmax (fp32, exact power-of-two
  * rescaling), P rounded to bf16 before PV, O rounded to bf16.
  *
  * Arguments, layouts, ownership and errors as nle_block_attn_fwd, without

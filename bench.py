@@ -76,7 +76,7 @@ NCU_TRAFFIC = {
                  "tensor_pipe_pct": 44.4},
     # posterior pooling over the whole batch-128 workload (58,903 frames)
     "posterior_pool": {"files": ('pool_sm100a.cu', 'nle_device.cuh'),
-                      "source_sha256": "377b218edef5a26471eb2a6eb04fe40a21a24780c34f4a3b9fcb1405a51f5f2a",
+                      "source_sha256": "9c30451e84816fe70b5bf4476faf488635d46f14fb73b2cdcfebbd7b1724dfca",
                       "traffic_over_algorithmic": (150827776 + 28794368) / 211398236},
     # CTC argmax: captured on 16 utterances (3,300 rows, 662.4 MB); traffic grows
     # with rows, so the ratio is applied to the full batch

@@ -11,10 +11,16 @@
 // sum taken about its own maximum, and a window divides e^{log w_t - max}
 // by its sum: no underflow when the blank dominates by far.
 //
-// One kernel, HBM-bound (reads each frame's hidden row and logits once,
-// writes each pooled row once).  A warp takes whole windows: it reduces each
-// frame's logits to the frame's log weight, then every lane forms 8 output
-// elements (16-byte chunks of the hidden dimension) at a time.
+// HBM-bound (reads each frame's hidden row and logits once, writes each
+// pooled row once).  A warp takes whole windows: it reduces each frame's
+// logits to the frame's log weight, then every lane forms 8 output elements
+// (16-byte chunks of the hidden dimension) at a time.  Two kernels:
+//   posterior_pool_pipe_kernel<NCH>  the encoder's shapes (windows of <= 2
+//                  frames, width <= 1024, <= 256 classes in 16-byte chunks):
+//                  two windows in flight per warp through a cp.async ring in
+//                  shared memory, offsets fixed at compile time for NCH
+//                  hidden chunks per lane, packed fp32 FMAs;
+//   posterior_pool_kernel  any other shape: loads in registers.
 #include <climits>
 
 #include "nle.h"

@@ -122,12 +122,53 @@ struct Params {
     uint32_t qk_bytes;  // QK stage
     uint32_t v_bytes;   // V stage
     uint32_t bars_off;  // barriers, after the QK and V rings
+    int split;          // one row tile per work item (batches that do not fill the GPU)
     float scale_log2;
     __nv_bfloat16 *out;
     int out_stride;     // elements between output frames (heads * 64)
     int32_t *status;
     unsigned long long wait_ns;
     int flags;
+};
+
+// The CTA's work items in order: raw item i = blockIdx.x + k * gridDim.x.
+// Whole items: i = b * H + h, both row tiles of block b, head h.  Split
+// items (p.split, for batches too small to fill the GPU): i = (b * H + h) *
+// 2 + x, row tile x alone, so the two row tiles of a block run on two
+// chains at once; a block of <= 128 frames has no row tile 1, and every
+// role skips that item alike.
+struct ItemSeq {
+    int b, h, x;      // the next raw item: block, head, row tile
+    int sb, sh, sx;   // the step gridDim.x in the same digits
+
+    __device__ __forceinline__ void init(const Params &p)
+    {
+        const int H = p.heads, G = (int)gridDim.x, i = (int)blockIdx.x;
+        const int bh = p.split ? i >> 1 : i, sbh = p.split ? G >> 1 : G;
+        x = p.split ? i & 1 : 0;
+        sx = p.split ? G & 1 : 0;
+        b = bh / H;
+        h = bh % H;
+        sb = sbh / H;
+        sh = sbh % H;
+    }
+
+    // the next raw item: block b, head h, row tile x (0 for whole items)
+    __device__ __forceinline__ void next(const Params &p, int &ob, int &oh, int &ox)
+    {
+        ob = b;
+        oh = h;
+        ox = x;
+        x += sx;
+        const int carry = x >> 1;   // x in {0, 1, 2}
+        x &= 1;
+        h += sh + carry;
+        b += sb;
+        if (h >= p.heads) {   // h < 2 H: one wrap at most
+            h -= p.heads;
+            ++b;
+        }
+    }
 };
 
 template <int NB>
@@ -189,10 +230,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bars->tmem_base;
     volatile int *abort_flag = &bars->abort_flag;
     const unsigned long long wait_ns = p.wait_ns;
-    const int H = p.heads;
-    // work items of this CTA: item = blockIdx.x + n * gridDim.x = b * H + h
-    const int step_b = (int)(gridDim.x / H), step_h = (int)(gridDim.x % H);
-    const int first_b = (int)(blockIdx.x / H), first_h = (int)(blockIdx.x % H);
 
     if (warp == 0 || warp == 1) {
         // ==================================================== producers
@@ -206,10 +243,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t pol = policy_evict_first();
         const bool skip0 = !is_v && (p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) != 0;
         int n = 0;   // items whose copies were issued
-        for (int b = first_b, h = first_h;; ++n) {
-            int f0, L, seq;
+        ItemSeq items;
+        items.init(p);
+        for (;;) {
+            int b, h, x, f0, L, seq;
+            items.next(p, b, h, x);
             if (!w.find(b, lane, f0, L, seq))
                 break;
+            if (x == 1 && L <= kQTile)
+                continue;   // split items: the block has no row tile 1
             const int s = n % nst;
             const uint32_t u = (uint32_t)(n / nst);
             if (u > 0 && !wait_bar(smem_u32(is_v ? &bars->v_empty[s] : &bars->qk_empty[s]), (u - 1) & 1, abort_flag,
@@ -221,25 +263,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(bar, p.B * kRowBytes);
                     tma_load_2d(v_base + s * p.v_bytes, &tm_v, h * 64, f0, bar, pol);
                 } else if (!(skip0 && n == 0)) {
-                    const bool two = L > kQTile;
+                    // Q of the item's row tiles (a split item: its one tile), then K
+                    const bool t0 = !p.split || x == 0;
+                    const bool t1 = p.split ? x == 1 : L > kQTile;
                     const uint32_t bar = smem_u32(&bars->qk_full[s]);
-                    const uint32_t bytes = (p.q0rows + (two ? p.q1rows : 0) + p.B) * kRowBytes;
+                    const uint32_t bytes = ((t0 ? p.q0rows : 0) + (t1 ? p.q1rows : 0) + p.B) * kRowBytes;
                     const uint32_t qdst = qk_base + s * p.qk_bytes;
                     mbar_arrive_expect_tx(bar, bytes);
-                    tma_load_2d(qdst, &tm_q0, h * 64, f0, bar, pol);
-                    if (two)
+                    if (t0)
+                        tma_load_2d(qdst, &tm_q0, h * 64, f0, bar, pol);
+                    if (t1)
                         tma_load_2d(qdst + kQTile * kRowBytes, &tm_q1, h * 64, f0 + kQTile, bar, pol);
                     tma_load_2d(qdst + p.q_bytes, &tm_k, h * 64, f0, bar, pol);
                 }
                 NLE_TRACE_AT(0, n, is_v ? 1 : 0);
             }
             __syncwarp();
-            b += step_b;
-            h += step_h;
-            if (h >= H) {
-                h -= H;
-                ++b;
-            }
+            ++n;
         }
         if (!is_v && w.bad && lane == 0)
             report(p.status, NLE_ERR_INVALID_ARG);
@@ -274,16 +314,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         PlanWalker w;
         w.init(p.cu, p.n_seq, p.total, p.B, lane);
         // the CTA's item sequence: item n is blockIdx.x + n * gridDim.x
-        int b = first_b, h = first_h;
+        ItemSeq items;
+        items.init(p);
         int next_n = 0;      // next item of the CTA's sequence (not yet looked at)
         int n = -1;          // current item
         int x = 1;           // current row tile of the item
+        bool fresh = false;  // the current unit is its item's first (its stages still to be waited for)
         uint32_t uses = 0;   // units (item, row tile) this slot has computed
         int f0 = 0, L = 0, hcur = 0, nkeys = 16, s = 0, sv = 0;
         bool ok = true;
 
         // Move to the slot's next unit: row tile 1 of the current item if it
-        // has one, else row tile 0 of the slot's next item.  The leader then
+        // has one (whole items), else the first (or, split, the only) row
+        // tile of the slot's next item.  The leader then
         // issues the unit's S MMA (after the slot's previous O has been read
         // by all four warps).  False at the end of the work.
         // Both ring depths are even, so the item's stages have the parity of
@@ -291,39 +334,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         // phases one by one, in order (a parity wait is only meaningful on
         // the current phase or the one after it).
         auto advance = [&]() -> bool {
-            if (!(x == 0 && L > kQTile)) {
+            if (p.split || !(x == 0 && L > kQTile)) {
                 // the slot's next item: pass over the other slot's one
                 for (;;) {
-                    int sf0, sL, sseq;
+                    int b, hh, xx, sf0, sL, sseq;
+                    items.next(p, b, hh, xx);
                     if (!w.find(b, lane, sf0, sL, sseq))
                         return false;
+                    if (xx == 1 && sL <= kQTile)
+                        continue;   // split items: the block has no row tile 1
                     const int nn = next_n++;
-                    const int hh = h;
-                    b += step_b;
-                    h += step_h;
-                    if (h >= H) {
-                        h -= H;
-                        ++b;
-                    }
                     if ((nn & 1) != t)
                         continue;
                     n = nn;
                     f0 = sf0;
                     L = sL;
                     hcur = hh;
+                    x = xx;
                     break;
                 }
-                x = 0;
+                fresh = true;
                 nkeys = (L + 15) & ~15;   // MMA extent over keys
                 s = n % p.sqk;
                 sv = n % p.nsv;
             } else {
                 x = 1;
+                fresh = false;
             }
             if (leader) {
                 if (lane == 0)
                     NLE_TRACE_AT(1 + t, n * 2 + x, 0);
-                if (x == 0 &&
+                if (fresh &&
                     !wait_bar(smem_u32(&bars->qk_full[s]), (uint32_t)(n / p.sqk) & 1, abort_flag, wait_ns, p.status)) {
                     ok = false;
                     return false;
@@ -345,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < 4; ++kk)
                         mma_ss(slot, da + 2 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
                     mma_commit(smem_u32(&bars->s_full[t]));
-                    if (x == 1 || L <= kQTile)   // the item's last S: its QK stage can be reused
+                    if (p.split || x == 1 || L <= kQTile)   // the item's last S: its QK stage can be reused
                         mma_commit(smem_u32(&bars->qk_empty[s]));
                     NLE_TRACE_AT(1 + t, n * 2 + x, 1);
                 }
@@ -398,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) {
                 if (!wait_bar(smem_u32(&bars->wg_p[t]), uses & 1, abort_flag, wait_ns, p.status))
                     break;
-                if (x == 0) {
+                if (fresh) {
                     if (!wait_bar(smem_u32(&bars->v_full[sv]), ph_v, abort_flag, wait_ns, p.status))
                         break;
                     if (L < nkeys && L < p.B) {
@@ -427,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_ts(slot + kOCol, slot + kk * 8, dv + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
                                kk > 0 ? 1u : 0u);
                     mma_commit(smem_u32(&bars->o_full[t]));
-                    if (x == 1 || L <= kQTile)   // the item's last PV: its V stage can be reused
+                    if (p.split || x == 1 || L <= kQTile)   // the item's last PV: its V stage can be reused
                         mma_commit(smem_u32(&bars->v_empty[sv]));
                     NLE_TRACE_AT(1 + t, n * 2 + x, 6);
                 }
@@ -613,10 +654,19 @@ extern "C" int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v
         !nle::encode_tmap_bf16_2d(&tv, v, cols, rows, stride, 64, B))
         return NLE_ERR_CUDA;
 
+    // Work split: a batch whose (block, head) items fit one per SM runs each
+    // row tile as its own item (two chains per block at once); blocks <=
+    // sum ceil(T_i / B) <= (T + n_seq (B - 1)) / B
+    const long long items_bound = (total_frames + (long long)n_seq * (B - 1)) / B * heads;
+    p.split = B > kQTile && (flags & NLE_FLAG_WHOLE_ITEMS) == 0 &&
+              ((flags & NLE_FLAG_SPLIT_ITEMS) != 0 || items_bound <= di.sm_count);
+    const long long work = p.split ? 2 * items_bound : max_items;
+    if (p.split && 2 * items_bound > 0x7fffffffLL)
+        return NLE_ERR_UNSUPPORTED;
     const KernelInfo kern = pick_kernel(NB);
     if (!nle::allow_max_dynamic_smem(reinterpret_cast<const void *>(kern.fn), dev, di.smem_optin))
         return NLE_ERR_CUDA;
-    const int grid = (int)(max_items < di.sm_count ? max_items : di.sm_count);
+    const int grid = (int)(work < di.sm_count ? work : di.sm_count);
     kern.fn<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(tq0, tq1, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? NLE_OK : NLE_ERR_CUDA;
 }

@@ -82,6 +82,8 @@ NLE_ERR_MISALIGNED = -3
 NLE_ERR_CUDA = -4
 NLE_ERR_TIMEOUT = -5
 NLE_FLAG_TEST_SKIP_FIRST_LOAD = 1
+NLE_FLAG_WHOLE_ITEMS = 2    # block attention: never run row tiles as separate items
+NLE_FLAG_SPLIT_ITEMS = 4    # block attention: always run row tiles as separate items
 
 
 class NLEError(RuntimeError):

@@ -82,6 +82,14 @@ typedef enum {
  * consumers' bounded waits expire and the kernel reports NLE_ERR_TIMEOUT.
  * Exercises the timeout path without hanging the GPU. */
 #define NLE_FLAG_TEST_SKIP_FIRST_LOAD 1
+/* Work split of nle_block_attn_fwd_ex (results are identical either way).
+ * By default a batch whose (block, head) items number at most the device's
+ * SM count runs each row tile of a block as its own work item, so the two
+ * 128-row tiles of a block run at once on two chains (lower latency for
+ * short batches, K and V read once per row tile); larger batches run whole
+ * items.  These flags force one or the other. */
+#define NLE_FLAG_WHOLE_ITEMS 2
+#define NLE_FLAG_SPLIT_ITEMS 4
 
 /* ABI version (NLE_ABI_VERSION of the build). */
 int nle_version(void);
@@ -116,7 +124,8 @@ int nle_block_attn_fwd(const void *q, const void *k, const void *v, void *out,
  * dev_status       device int32 or NULL; receives the first in-kernel error
  *                  (NLE_ERR_TIMEOUT or NLE_ERR_INVALID_ARG); never reset by
  *                  the library.
- * flags            NLE_FLAG_* (test hooks only; 0 in production)
+ * flags            NLE_FLAG_* (0 in production: the test hook, and the
+ *                  work-split overrides)
  * wait_limit_ns    limit of every in-kernel wait; 0 selects 1 s.
  */
 int nle_block_attn_fwd_ex(const void *q, const void *k, const void *v,

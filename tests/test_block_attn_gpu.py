@@ -299,3 +299,34 @@ def test_concurrent_launches_on_two_streams(cuda_device):
     torch.cuda.synchronize()
     for x, out in zip(xs, outs):
         _compare(out, oracle.block_attn(x["q"], x["k"], x["v"], x["cu"], block_frames=200))
+
+
+@pytest.mark.parametrize("B,lengths,heads", [
+    (200, [400], 8),                          # config 1's shape: split by default
+    (200, [800], 16),                         # config 2's shape
+    (200, [201, 200, 199, 128, 129, 1, 0, 55, 350], 4),
+    (129, [129, 130, 258, 400, 7], 3),
+    (256, [256, 512, 300, 129, 128, 1000], 4),
+    (200, list(wl.draw_lengths(4)[:20]), 16),  # whole items by default (320+ items)
+])
+def test_work_split_bit_equal(B, lengths, heads, cuda_device):
+    """Row tiles as separate work items (split) and whole (block, head) items
+    compute the same numbers bit for bit: each row tile's S, softmax, PV and
+    output are the same instructions on the same data, only the CTA and
+    chain that run them change.  Both are also within tolerance of the
+    oracle."""
+    nle = _nle()
+    x = wl.block_inputs(lengths=lengths, heads=heads, seed=B + len(lengths))
+    q, k, v = (x[n].to(cuda_device) for n in ("q", "k", "v"))
+    cu = torch.from_numpy(x["cu"]).to(cuda_device)
+    outs = {}
+    for name, flags in (("whole", nle.NLE_FLAG_WHOLE_ITEMS), ("split", nle.NLE_FLAG_SPLIT_ITEMS), ("auto", 0)):
+        out = torch.full_like(q, float("nan"))
+        status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+        nle.nle_block_attn_fwd_ex(q, k, v, out, cu, block_frames=B, dev_status=status, flags=flags)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        outs[name] = out
+    assert torch.equal(outs["split"], outs["whole"])
+    assert torch.equal(outs["auto"], outs["whole"])
+    _compare(outs["split"], oracle.block_attn(x["q"], x["k"], x["v"], x["cu"], B))

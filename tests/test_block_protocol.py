@@ -140,3 +140,19 @@ def test_model_catches_a_stage_shared_by_both_warpgroups():
         with pytest.raises(AssertionError, match="parity wait"):
             _simulate(lengths, 2, 3, seed, p_complete=0.05, p_out_of_order=1.0)
         _simulate(lengths, 2, 4, seed, p_complete=0.05, p_out_of_order=1.0)   # even ring: fine
+
+
+def test_split_items_meet_the_protocol():
+    """Split work items (one row tile each, for batches that do not fill the
+    GPU) meet the protocol as items of at most 128 rows: a block of L > 128
+    frames becomes two items, of 128 and L - 128 rows."""
+    rng = random.Random(77)
+    for trial in range(200):
+        blocks = [rng.choice([200, 193, 150, 129, 128, 100, 40, 1]) for _ in range(rng.randint(1, 10))]
+        items = []
+        for L in blocks:
+            items.append(min(L, 128))
+            if L > 128:
+                items.append(L - 128)
+        _simulate(items, 2, 4, trial)
+        _simulate(items, 2, 2, trial, p_complete=0.05, p_out_of_order=1.0)

@@ -68,12 +68,14 @@ NCU_TRAFFIC = {
                    "traffic_over_algorithmic": (345912064 + 88160512) / 439304192,
                    "tensor_pipe_pct": 27.2},
     # fused projection + block attention on the batch-128 workload (d_model 1024,
-    # 16 heads); DRAM writes sit below the output's bytes because part of it is
-    # still in L2 when the kernel ends
+    # 16 heads); X is read from DRAM about four times (the CTAs of the 16 heads
+    # reach a row at different times and X is about the size of L2), and DRAM
+    # writes sit below the output's bytes because part of it is still in L2
+    # when the kernel ends
     "qkv_attn": {"files": ('qkv_attn_sm100a.cu', 'attn_softmax.cuh', 'nle_device.cuh'),
-                 "source_sha256": "2a9ce094c52f98fff402b83e264ef9084cdbfed03fd19d434410850bcb92aff0",
-                 "traffic_over_algorithmic": (127470592 + 82170624) / 247564288,
-                 "tensor_pipe_pct": 44.4},
+                 "source_sha256": "6cf4f4b5b448092c88c5f08d7fdf1ac3700dc546ffb1959819c0fe2b3f61e9ee",
+                 "traffic_over_algorithmic": (511541248 + 110533632) / 247564288,
+                 "tensor_pipe_pct": 38.5},
     # posterior pooling over the whole batch-128 workload (58,903 frames)
     "posterior_pool": {"files": ('pool_sm100a.cu', 'nle_device.cuh'),
                       "source_sha256": "9c30451e84816fe70b5bf4476faf488635d46f14fb73b2cdcfebbd7b1724dfca",

@@ -13,40 +13,45 @@
 // of the linear layer's weight W [3*H*64][D] (output features x input
 // features), and b the optional bias.  Q, K and V never leave the SM.
 //
-// Design (one persistent CTA per SM, 12 warps; work item = (block, head),
-// dealt round-robin over the CTAs like the block kernel):
-//   warp 0      TMA producer: walks the plan, writes each item's descriptor
-//               into a small ring, and streams the projection operands in
-//               stages of 64 input features: the row tile's X box (128 rows
-//               x 64) and the head's three 64-row W boxes (192 x 64), all
-//               128-byte swizzled, no multicast.  Row tile 0 is block rows
-//               0..127, row tile 1 (blocks longer than 128 frames) rows
-//               128..255.
+// Work split: the (head, frame) positions h * T + f are cut into one equal
+// range per CTA; a CTA takes the (block, head) items whose first position
+// lies in its range, so its items form runs of consecutive blocks of one
+// head (one run, two where the range crosses a head).  The blocks of a run
+// cover consecutive frames, so the run's projection is a plain row range of
+// X: it is computed in tiles of 128 consecutive frames, whatever the block
+// boundaries, and only the last tile of a run is ragged.
+//
+// Design (one persistent CTA per SM, 12 warps):
+//   warp 0      walks the CTA's items, writes each block's descriptor into
+//               one ring and each projection tile's into another, and
+//               streams the projection operands in stages of 64 input
+//               features: the tile's X box (128 frames x 64) and the head's
+//               three 64-row W boxes (192 x 64), 128-byte swizzled, no
+//               multicast.
 //   warp 1      owns TMEM and issues the projection MMAs (lane 0):
 //               D[128 x 192] += X_tile W_h^T, tcgen05.mma kind::f16, M=128,
 //               N=192, K=16 x 4 per stage, fp32 accumulator in TMEM
 //               columns 0..191.
-//   warps 4-7   projection epilogue: per row (TMEM lane) reads D, adds the
-//               bias (fetched into shared memory when the item starts),
-//               rounds to bf16 and writes the row's q into TMEM (columns
-//               192 + 32 x, bf16 pairs: the A operand of the S MMA) and its k
-//               and v into shared memory in the layouts the attention MMAs
-//               read (K K-major, V N-major, 128-byte swizzle); rows at or
-//               past the block end are written as zeros.  Then D is released
-//               for the next row tile's projection.
+//   warps 4-7   projection epilogue: each lane reads its frame's 192 columns
+//               of D (+ bias), rounds them to bf16 in registers and releases
+//               D at once, so the next tile's projection starts; it then
+//               writes the row's q, k and v into the shared-memory buffers
+//               of the block the frame belongs to (K-major Q and K, N-major
+//               V, 128-byte swizzle), and hands a block to the attention
+//               when its last frame is written.
 //   warps 8-11  attention, as one tile warpgroup of the block kernel, on
-//               TMEM columns 256..511: S = Q_x K^T (M=128, N=ceil16(L), A
-//               from TMEM), fp32 register softmax with one shift per row, P
-//               (bf16) over S, O = P V (P from TMEM), O / rowsum rounded to
-//               bf16 and written with 16-byte stores; rows past the block
-//               end are never written.
-// The projection of the next item runs in its own TMEM columns while the
-// current item's attention runs.  There is one set of Q/K/V buffers: the
-// epilogue of the next item's first row tile stores Q and K once the current
-// item's last S MMA has completed, holds V in registers and releases D (so
-// the next row tile's projection starts), and stores V once the current
-// item's last PV has completed.  With Q in TMEM, shared memory holds K, V
-// and four 40 KB stages (B <= 256).
+//               TMEM columns 256..511: S = Q_x K^T (M=128, N=ceil16(L)), fp32
+//               register softmax with one shift per row, P (bf16) over S,
+//               O = P V (P from TMEM), O / rowsum rounded to bf16 and written
+//               with 16-byte stores; rows past the block end are never
+//               written.
+// There is one Q/K buffer and two V buffers: the epilogue stores the q and
+// k rows of a block once the previous block's last S MMA has completed, and
+// its v rows once the last PV of the block two before has completed (blocks
+// alternate between the V buffers); V rows L..ceil16(L)-1 (read by the PV
+// MMA, weighted by zeros) are cleared.  Shared memory: Q (max(ceil16(B),
+// 128) rows), K and two V buffers (ceil16(B) rows each) and three 40 KB
+// stages for B = 200.
 //
 // Every mbarrier wait is bounded (see nle_device.cuh); on expiry the CTA
 // drains its copies and MMAs in flight, frees TMEM and returns.
@@ -57,26 +62,6 @@
 #include "nle_device.cuh"
 #include "nle_host.h"
 
-// Optional cycle trace of CTA 0 for performance analysis (not built by
-// default): QKV_TRACE_AT(role, item, event) stores clock64() into a device
-// buffer registered with nle_qkv_trace_set().
-#ifdef NLE_TRACE
-__device__ unsigned long long *g_qkv_trace = nullptr;
-extern "C" int nle_qkv_trace_set(void *p)
-{
-    return cudaMemcpyToSymbol(g_qkv_trace, &p, sizeof(p)) == cudaSuccess ? 0 : -1;
-}
-#define QKV_TRACE_AT(role, n, ev)                                                                       \
-    do {                                                                                                \
-        if (blockIdx.x == 0 && g_qkv_trace && (n) < 64)                                                 \
-            g_qkv_trace[((role) * 64 + (n)) * 16 + (ev)] = clock64();                                   \
-    } while (0)
-#else
-#define QKV_TRACE_AT(role, n, ev) \
-    do {                          \
-    } while (0)
-#endif
-
 namespace {
 
 using namespace nle;
@@ -85,38 +70,48 @@ constexpr int kThreads = 384;
 constexpr int kEpi0 = 4;           // warps 4-7: projection epilogue
 constexpr int kAttn0 = 8;          // warps 8-11: attention
 constexpr int kSeg = 64;
-constexpr int kQTile = 128;
+constexpr int kQTile = 128;        // attention row tile
+constexpr int kPTile = 128;        // projection tile: consecutive frames
 constexpr int kRowBytes = 128;     // one frame of one head: 64 bf16
 constexpr uint32_t kXBytes = 128 * 128;          // X box: 128 rows x 64 features
 constexpr uint32_t kWBytes = 192 * 128;          // W boxes: 192 rows x 64 features
 constexpr uint32_t kStageBytes = kXBytes + kWBytes;
 constexpr int kMaxStages = 4;
 constexpr int kDescRing = 8;
-constexpr uint32_t kDescReaders = 9;             // warp 1, epilogue and attention warps
+constexpr uint32_t kBlockReaders = 8;            // epilogue and attention warps
+constexpr uint32_t kTileReaders = 5;             // warp 1 and the epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kDCol = 0;      // projection accumulator, 192 columns
 constexpr uint32_t kSCol = 256;    // attention: S (<= 256 columns), P over S, O at +128
 constexpr uint32_t kOCol = 128;
-constexpr uint32_t kQCol = 192;    // Q of row tile x (bf16 pairs, 32 columns) at 192 + 32 x
 
-struct ItemDesc {
-    int f0, L, h, pad;
+// A block (f0, L, head, run) or a projection tile (first frame, 1, head,
+// run); L < 0 ends a ring.
+struct Desc {
+    int f0, L, h, run;
 };
 
 struct Bars {
     uint64_t st_full[kMaxStages];
     uint64_t st_empty[kMaxStages];   // the stage's MMAs have completed
-    uint64_t d_full;                 // the row tile's projection has completed
+    uint64_t d_full;                 // the tile's projection has completed
     uint64_t d_empty;                // 4 arrivals: the epilogue has read D
-    uint64_t qkv_ready;              // 4 arrivals: the item's Q, K, V are in shared memory
-    uint64_t qk_free;                // the item's last S MMA has completed (Q and K read)
-    uint64_t v_free;                 // the item's last PV MMA has completed (V read)
-    uint64_t desc_full[kDescRing];
-    uint64_t desc_empty[kDescRing];  // every reader has read the entry
+    uint64_t qkv_ready;              // 4 arrivals: a block's Q, K, V are in shared memory
+    uint64_t qk_free;                // the block's last S MMA has completed (Q and K read)
+    uint64_t v_free[2];              // per V buffer: a block's last PV MMA has completed (V read)
+    uint64_t blk_full[kDescRing];
+    uint64_t blk_empty[kDescRing];   // every reader has read the entry
+    uint64_t tile_full[kDescRing];
+    uint64_t tile_empty[kDescRing];
     uint64_t s_full, wg_p, o_full, wg_o;
     uint64_t mma_done[2];
-    ItemDesc desc[kDescRing];
-    uint4 bias[4][24];               // the current item's 192 bias values, one copy per epilogue warp
+    Desc blk[kDescRing];
+    Desc tile[kDescRing];
+    // the q, k and v bias rows of a run's head, by run parity: every
+    // epilogue warp writes the copy of a run before its first tile (the same
+    // values) and reads it through the run; the warps are less than one
+    // tile apart, so no warp still reads a copy when it is rewritten
+    uint4 bias[2][24];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -129,7 +124,7 @@ struct Params {
     int B;            // block_frames
     int ksteps;       // input features / 64
     int nst;          // stage ring depth
-    uint32_t v_off, st_off, bars_off;   // K at 0, then V, stages, barriers
+    uint32_t k_off, v_off, v_size, st_off, bars_off;   // Q at 0, then K, V0, V1, stages, barriers
     const __nv_bfloat16 *bias;   // nullable, [3 * heads * 64]
     float scale_log2;
     __nv_bfloat16 *out;
@@ -153,11 +148,34 @@ __device__ __forceinline__ uint64_t policy_evict_normal()
     return p;
 }
 
+// The first unit whose first frame is >= F (units tile the utterances'
+// frames in order; utterances flagged invalid by the walker hold none), or
+// the number of units when there is none.  Queries must not decrease.
+__device__ __forceinline__ long long first_unit_from(PlanWalker &w, int F, int lane)
+{
+    for (;;) {
+        const bool in = w.base + lane < w.n_seq && w.len > 0 && w.start + w.len > F;
+        const unsigned m = __ballot_sync(kFull, in);
+        if (m) {
+            const int src = __ffs(m) - 1;
+            const int incl_s = __shfl_sync(kFull, w.incl, src);
+            const int st = __shfl_sync(kFull, w.start, src);
+            const int nb = __shfl_sync(kFull, w.units, src);
+            const int j = F <= st ? 0 : (F - st + w.unit - 1) / w.unit;   // may be nb: the next utterance
+            return (long long)w.before + (incl_s - nb) + j;
+        }
+        if (w.base + 32 >= w.n_seq)
+            return (long long)w.before + w.group_units;
+        w.before += w.group_units;
+        w.base += 32;
+        w.load_group(lane);
+    }
+}
+
 // 64 fp32 accumulator columns of this lane's row (+ bias), rounded to bf16
-// pairs in `pk` (zeros when the row lies at or past the block end).  The
-// TMEM loads are warp-collective: every lane of the warp calls this,
-// whatever its row.
-__device__ __forceinline__ void epi_load(uint32_t taddr, const uint4 *bias, bool valid, uint32_t (&pk)[32])
+// pairs in `pk`.  The TMEM loads are warp-collective: every lane of the warp
+// calls this.
+__device__ __forceinline__ void epi_load(uint32_t taddr, const uint4 *bias, uint32_t (&pk)[32])
 {
     uint32_t v[64];
     tmem_ld32_nowait(taddr, &v[0]);
@@ -184,9 +202,8 @@ __device__ __forceinline__ void epi_load(uint32_t taddr, const uint4 *bias, bool
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-            pk[4 * c + e] = valid ? pack_bf16x2(__uint_as_float(v[8 * c + 2 * e]) + b[2 * e],
-                                                __uint_as_float(v[8 * c + 2 * e + 1]) + b[2 * e + 1])
-                                  : 0u;
+            pk[4 * c + e] = pack_bf16x2(__uint_as_float(v[8 * c + 2 * e]) + b[2 * e],
+                                        __uint_as_float(v[8 * c + 2 * e + 1]) + b[2 * e + 1]);
     }
 }
 
@@ -207,9 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t k_base = smem_u32(smem);
-    const uint32_t v_base = k_base + p.v_off;
-    const uint32_t st_base = k_base + p.st_off;
+    const uint32_t q_base = smem_u32(smem);
+    const uint32_t k_base = q_base + p.k_off;
+    const uint32_t v_base = q_base + p.v_off;
+    const uint32_t st_base = q_base + p.st_off;
     Bars *bars = reinterpret_cast<Bars *>(smem + p.bars_off);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -224,10 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(&bars->d_empty), 4);
         mbar_init(smem_u32(&bars->qkv_ready), 4);
         mbar_init(smem_u32(&bars->qk_free), 1);
-        mbar_init(smem_u32(&bars->v_free), 1);
+        mbar_init(smem_u32(&bars->v_free[0]), 1);
+        mbar_init(smem_u32(&bars->v_free[1]), 1);
         for (int j = 0; j < kDescRing; ++j) {
-            mbar_init(smem_u32(&bars->desc_full[j]), 1);
-            mbar_init(smem_u32(&bars->desc_empty[j]), kDescReaders);
+            mbar_init(smem_u32(&bars->blk_full[j]), 1);
+            mbar_init(smem_u32(&bars->blk_empty[j]), kBlockReaders);
+            mbar_init(smem_u32(&bars->tile_full[j]), 1);
+            mbar_init(smem_u32(&bars->tile_empty[j]), kTileReaders);
         }
         mbar_init(smem_u32(&bars->s_full), 1);
         mbar_init(smem_u32(&bars->wg_p), 4);
@@ -255,89 +276,115 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int H = p.heads;
     const int KS = p.ksteps;
 
-    // every reader of the descriptor ring: entry of item n, then release it
-    auto read_desc = [&](int n, ItemDesc &d) -> bool {
+    // every reader of a descriptor ring: entry n, then release it
+    auto read_ring = [&](uint64_t *full, uint64_t *empty, const Desc *ring, int n, Desc &d) -> bool {
         const int j = n % kDescRing;
-        if (!wait_bar(smem_u32(&bars->desc_full[j]), (uint32_t)(n / kDescRing) & 1, abort_flag, wait_ns, p.status))
+        if (!wait_bar(smem_u32(&full[j]), (uint32_t)(n / kDescRing) & 1, abort_flag, wait_ns, p.status))
             return false;
-        d = bars->desc[j];
+        d = ring[j];
         __syncwarp();
         if (lane == 0)
-            mbar_arrive(smem_u32(&bars->desc_empty[j]));
+            mbar_arrive(smem_u32(&empty[j]));
         return true;
     };
 
     if (warp == 0) {
         // ==================================================== producer
-        const int step_b = (int)(gridDim.x / H), step_h = (int)(gridDim.x % H);
-        PlanWalker w;
-        w.init(p.cu, p.n_seq, p.total, p.B, lane);
-        const uint64_t pol_x = policy_evict_normal();   // X tiles: read by every head of the block
-        const uint64_t pol_w = policy_evict_last();     // W: read by every item
+        const uint64_t pol_x = policy_evict_normal();   // X rows: read by the CTAs of every head
+        const uint64_t pol_w = policy_evict_last();     // W: read by every tile
         const bool skip0 = (p.flags & NLE_FLAG_TEST_SKIP_FIRST_LOAD) != 0;
-        uint32_t g = 0;   // stages issued
-        int n = 0;        // items published
+        uint32_t g = 0;        // stages issued
+        int nblk = 0, ntile = 0;
         bool ok = true;
-        auto publish = [&](const ItemDesc &d) -> bool {
+        auto publish = [&](uint64_t *full, uint64_t *empty, Desc *ring, int &n, const Desc &d) -> bool {
             const int j = n % kDescRing;
-            if (n >= kDescRing && !wait_bar(smem_u32(&bars->desc_empty[j]), (uint32_t)(n / kDescRing - 1) & 1,
-                                            abort_flag, wait_ns, p.status))
+            if (n >= kDescRing && !wait_bar(smem_u32(&empty[j]), (uint32_t)(n / kDescRing - 1) & 1, abort_flag,
+                                            wait_ns, p.status))
                 return false;
             if (lane == 0) {
-                bars->desc[j] = d;
-                mbar_arrive(smem_u32(&bars->desc_full[j]));
+                ring[j] = d;
+                mbar_arrive(smem_u32(&full[j]));
             }
             __syncwarp();
+            ++n;
             return true;
         };
-        for (int b = (int)(blockIdx.x / H), h = (int)(blockIdx.x % H);; ++n) {
-            int f0, L, seq;
-            if (!w.find(b, lane, f0, L, seq))
-                break;
-            if (!publish(ItemDesc{f0, L, h, 0})) {
-                ok = false;
-                break;
+        // one projection tile: its descriptor, then its KS stages
+        auto issue_tile = [&](int t0, int h, int run) -> bool {
+            if (!publish(bars->tile_full, bars->tile_empty, bars->tile, ntile, Desc{t0, 1, h, run}))
+                return false;
+            for (int kb = 0; kb < KS; ++kb, ++g) {
+                const int s = (int)(g % (uint32_t)p.nst);
+                const uint32_t u = g / (uint32_t)p.nst;
+                if (u > 0 && !wait_bar(smem_u32(&bars->st_empty[s]), (u - 1) & 1, abort_flag, wait_ns, p.status))
+                    return false;
+                if (lane == 0 && !(skip0 && g == 0)) {
+                    const uint32_t bar = smem_u32(&bars->st_full[s]);
+                    const uint32_t dst = st_base + (uint32_t)s * kStageBytes;
+                    mbar_arrive_expect_tx(bar, kStageBytes);
+                    tma_load_2d(dst, &tm_x, kb * 64, t0, bar, pol_x);
+                    tma_load_2d(dst + kXBytes, &tm_w, kb * 64, h * 64, bar, pol_w);
+                    tma_load_2d(dst + kXBytes + 8192, &tm_w, kb * 64, (H + h) * 64, bar, pol_w);
+                    tma_load_2d(dst + kXBytes + 16384, &tm_w, kb * 64, (2 * H + h) * 64, bar, pol_w);
+                }
+                __syncwarp();
             }
-            const int tiles = L > kQTile ? 2 : 1;
-            if (lane == 0)
-                QKV_TRACE_AT(0, n, 0);
-            for (int x = 0; x < tiles && ok; ++x) {
-                for (int kb = 0; kb < KS; ++kb, ++g) {
-                    const int s = (int)(g % (uint32_t)p.nst);
-                    const uint32_t u = g / (uint32_t)p.nst;
-                    if (u > 0 && !wait_bar(smem_u32(&bars->st_empty[s]), (u - 1) & 1, abort_flag, wait_ns, p.status)) {
+            return true;
+        };
+
+        // this CTA's positions [lo, hi) of the H * total (head, frame) positions
+        const long long HT = (long long)H * p.total;
+        const long long lo = HT * (long long)blockIdx.x / (long long)gridDim.x;
+        const long long hi = HT * ((long long)blockIdx.x + 1) / (long long)gridDim.x;
+        int bad = 0;
+        if (lo < hi) {
+            int h = (int)(lo / p.total);
+            PlanWalker w;
+            w.init(p.cu, p.n_seq, p.total, p.B, lane);
+            long long u = first_unit_from(w, (int)(lo % p.total), lane);
+            int run = -1, run_h = -1, run_end = 0, next_t = 0;
+            for (;;) {
+                int f0, L, seq;
+                if (!w.find(u, lane, f0, L, seq)) {
+                    // past the last block of head h: the next head from its first block
+                    bad |= w.bad;
+                    if (++h >= H || (long long)h * p.total >= hi)
+                        break;
+                    w.init(p.cu, p.n_seq, p.total, p.B, lane);
+                    u = 0;
+                    continue;
+                }
+                if ((long long)h * p.total + f0 >= hi)
+                    break;
+                // a run: consecutive blocks of one head over consecutive frames
+                if (h != run_h || f0 != run_end) {
+                    ++run;
+                    run_h = h;
+                    next_t = f0;
+                }
+                run_end = f0 + L;
+                if (!publish(bars->blk_full, bars->blk_empty, bars->blk, nblk, Desc{f0, L, h, run})) {
+                    ok = false;
+                    break;
+                }
+                // the tiles that hold this block's frames
+                for (; next_t < run_end; next_t += kPTile)
+                    if (!issue_tile(next_t, h, run)) {
                         ok = false;
                         break;
                     }
-                    if (lane == 0 && !(skip0 && g == 0)) {
-                        const uint32_t bar = smem_u32(&bars->st_full[s]);
-                        const uint32_t dst = st_base + (uint32_t)s * kStageBytes;
-                        mbar_arrive_expect_tx(bar, kStageBytes);
-                        tma_load_2d(dst, &tm_x, kb * 64, f0 + x * kQTile, bar, pol_x);
-                        tma_load_2d(dst + kXBytes, &tm_w, kb * 64, h * 64, bar, pol_w);
-                        tma_load_2d(dst + kXBytes + 8192, &tm_w, kb * 64, (H + h) * 64, bar, pol_w);
-                        tma_load_2d(dst + kXBytes + 16384, &tm_w, kb * 64, (2 * H + h) * 64, bar, pol_w);
-                        if (kb == 0)
-                            QKV_TRACE_AT(0, n, 1 + x);
-                        if (kb == KS - 1)
-                            QKV_TRACE_AT(0, n, 3 + x);
-                    }
-                    __syncwarp();
-                }
+                if (!ok)
+                    break;
+                ++u;
             }
-            if (!ok)
-                break;
-            b += step_b;
-            h += step_h;
-            if (h >= H) {
-                h -= H;
-                ++b;
-            }
+            bad |= w.bad;
         }
-        if (w.bad && lane == 0)
+        if (bad && lane == 0)
             report(p.status, NLE_ERR_INVALID_ARG);
-        if (ok)
-            publish(ItemDesc{0, -1, 0, 0});   // end marker
+        if (ok) {   // end markers
+            publish(bars->blk_full, bars->blk_empty, bars->blk, nblk, Desc{0, -1, 0, -1});
+            publish(bars->tile_full, bars->tile_empty, bars->tile, ntile, Desc{0, -1, 0, -1});
+        }
         // drain: the last copies of every stage must land before the CTA exits
         if (lane == 0) {
             const uint32_t nst = (uint32_t)p.nst;
@@ -351,49 +398,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t id_p = idesc_bf16_f32(128, 192, false);
         uint32_t g = 0, tiles_done = 0;
         for (int n = 0;; ++n) {
-            ItemDesc d;
-            if (!read_desc(n, d) || d.L < 0)
+            Desc d;
+            if (!read_ring(bars->tile_full, bars->tile_empty, bars->tile, n, d) || d.L < 0)
                 break;
-            const int tiles = d.L > kQTile ? 2 : 1;
+            if (tiles_done > 0 &&
+                !wait_bar(smem_u32(&bars->d_empty), (tiles_done - 1) & 1, abort_flag, wait_ns, p.status))
+                break;
+            tc_fence_after();
             bool ok = true;
-            for (int x = 0; x < tiles && ok; ++x) {
-                if (tiles_done > 0 &&
-                    !wait_bar(smem_u32(&bars->d_empty), (tiles_done - 1) & 1, abort_flag, wait_ns, p.status)) {
+            for (int kb = 0; kb < KS; ++kb, ++g) {
+                const int s = (int)(g % (uint32_t)p.nst);
+                if (!wait_bar(smem_u32(&bars->st_full[s]), (g / (uint32_t)p.nst) & 1, abort_flag, wait_ns,
+                              p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (lane == 0)
-                    QKV_TRACE_AT(1, n, 3 * x);
-                for (int kb = 0; kb < KS; ++kb, ++g) {
-                    const int s = (int)(g % (uint32_t)p.nst);
-                    if (!wait_bar(smem_u32(&bars->st_full[s]), (g / (uint32_t)p.nst) & 1, abort_flag, wait_ns,
-                                  p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    if (lane == 0 && kb == 0)
-                        QKV_TRACE_AT(1, n, 3 * x + 1);
-                    tc_fence_after();
-                    const uint32_t a = st_base + (uint32_t)s * kStageBytes;
-                    const uint64_t da = smem_desc_sw128(a, 16, 1024);
-                    const uint64_t db = smem_desc_sw128(a + kXBytes, 16, 1024);
-                    if (lane == 0) {
+                const uint32_t a = st_base + (uint32_t)s * kStageBytes;
+                const uint64_t da = smem_desc_sw128(a, 16, 1024);
+                const uint64_t db = smem_desc_sw128(a + kXBytes, 16, 1024);
+                if (lane == 0) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ss(tmem + kDCol, da + 2 * kk, db + 2 * kk, id_p, (kb | kk) ? 1u : 0u);
-                        mma_commit(smem_u32(&bars->st_empty[s]));
-                        if (kb == KS - 1) {
-                            mma_commit(smem_u32(&bars->d_full));
-                            QKV_TRACE_AT(1, n, 3 * x + 2);
-                        }
-                    }
-                    __syncwarp();
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tmem + kDCol, da + 2 * kk, db + 2 * kk, id_p, (kb | kk) ? 1u : 0u);
+                    mma_commit(smem_u32(&bars->st_empty[s]));
+                    if (kb == KS - 1)
+                        mma_commit(smem_u32(&bars->d_full));
                 }
-                ++tiles_done;
+                __syncwarp();
             }
             if (!ok)
                 break;
+            ++tiles_done;
         }
         if (lane == 0) {
             mma_commit(smem_u32(&bars->mma_done[0]));
@@ -404,84 +440,95 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ==================================================== projection epilogue
         const int qq = warp & 3;
         const uint32_t tD = tmem + kDCol + ((uint32_t)(qq * 32) << 16);
-        const uint32_t tQ = tmem + kQCol + ((uint32_t)(qq * 32) << 16);
-        const int NBr = ((p.B + 15) / 16) * 16;   // K and V rows the attention MMAs may read
-        uint4 *wbias = bars->bias[qq];
         uint32_t tiles_done = 0;
-        for (int n = 0;; ++n) {
-            ItemDesc d;
-            if (!read_desc(n, d) || d.L < 0)
+        int bias_run = -1;
+        int nb = 0;              // blocks handed to the attention
+        int tn = 0, bn = 0;      // descriptors read
+        Desc cb{0, -1, 0, -1};   // the block being filled
+        bool have = false, claimed = false;
+        bool ok = true;
+        for (;;) {
+            Desc td;
+            if (!read_ring(bars->tile_full, bars->tile_empty, bars->tile, tn++, td)) {
+                ok = false;
                 break;
-            // this item's q, k and v bias rows, fetched while its projection
-            // runs (off the path from the finished projection to the release
-            // of D)
-            if (p.bias && lane < 24)
-                wbias[lane] = __ldg(reinterpret_cast<const uint4 *>(p.bias + (size_t)((lane >> 3) * H + d.h) * 64) +
-                                    (lane & 7));
-            __syncwarp();
-            const uint4 *bq = p.bias ? wbias : nullptr;
-            const uint4 *bk = p.bias ? wbias + 8 : nullptr;
-            const uint4 *bv = p.bias ? wbias + 16 : nullptr;
-            const int tiles = d.L > kQTile ? 2 : 1;
-            bool ok = true;
-            for (int x = 0; x < tiles; ++x) {
-                if (!wait_bar(smem_u32(&bars->d_full), tiles_done & 1, abort_flag, wait_ns, p.status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (warp == kEpi0 && lane == 0)
-                    QKV_TRACE_AT(2, n, 5 * x);
-                const int r = x * kQTile + qq * 32 + lane;   // block row of this lane
-                const bool valid = r < d.L;
-                // every lane runs the (warp-collective) TMEM loads and
-                // stores; only rows inside the buffers are stored to shared
-                // memory.  The previous item's attention still reads the
-                // buffers: Q (TMEM columns 192..255) and K until its last S
-                // MMA has completed, V until its last PV.  V is held in
-                // registers meanwhile, so D is released for the next row
-                // tile's projection without waiting for that PV.
-                const bool first_tile_of_later_item = x == 0 && n > 0;
-                if (first_tile_of_later_item &&
-                    !wait_bar(smem_u32(&bars->qk_free), (uint32_t)(n - 1) & 1, abort_flag, wait_ns, p.status)) {
-                    ok = false;
-                    break;
-                }
-                if (warp == kEpi0 && lane == 0)
-                    QKV_TRACE_AT(2, n, 5 * x + 1);
-                {
-                    uint32_t pk[32];
-                    epi_load(tD, bq, valid, pk);
-                    tmem_st32(tQ + 32 * x, pk);   // Q: the A operand of the S MMA, from TMEM
-                    epi_load(tD + 64, bk, valid, pk);
-                    if (r < NBr)
-                        epi_store(pk, smem + (size_t)r * kRowBytes, r);
-                }
-                uint32_t pv[32];
-                epi_load(tD + 128, bv, valid, pv);
-                tmem_wait_st();
-                tc_fence_before();
+            }
+            if (td.L < 0)
+                break;
+            if (!wait_bar(smem_u32(&bars->d_full), tiles_done & 1, abort_flag, wait_ns, p.status))
+                break;
+            tc_fence_after();
+            // this lane's frame of the tile: its q, k and v, then D is free
+            uint32_t pq[32], pk[32], pv[32];
+            uint4 *rbias = bars->bias[td.run & 1];
+            if (p.bias && td.run != bias_run) {
+                if (lane < 24)
+                    rbias[lane] = __ldg(reinterpret_cast<const uint4 *>(p.bias + (size_t)((lane >> 3) * H + td.h) * 64) +
+                                        (lane & 7));
                 __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(smem_u32(&bars->d_empty));
-                if (warp == kEpi0 && lane == 0)
-                    QKV_TRACE_AT(2, n, 5 * x + 2);
-                if (first_tile_of_later_item &&
-                    !wait_bar(smem_u32(&bars->v_free), (uint32_t)(n - 1) & 1, abort_flag, wait_ns, p.status)) {
+                bias_run = td.run;
+            }
+            epi_load(tD, p.bias ? rbias : nullptr, pq);
+            epi_load(tD + 64, p.bias ? rbias + 8 : nullptr, pk);
+            epi_load(tD + 128, p.bias ? rbias + 16 : nullptr, pv);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bars->d_empty));
+            ++tiles_done;
+            const int f = td.f0 + qq * 32 + lane;
+            // the blocks of this run that hold frames of the tile, in order
+            for (;;) {
+                if (!have) {
+                    if (!read_ring(bars->blk_full, bars->blk_empty, bars->blk, bn++, cb)) {
+                        ok = false;
+                        break;
+                    }
+                    have = true;
+                    claimed = false;
+                }
+                if (cb.L < 0 || cb.run != td.run || cb.f0 >= td.f0 + kPTile)
+                    break;   // it starts in a later tile
+                const int r = f - cb.f0;
+                const bool mine = r >= 0 && r < cb.L;
+                // the previous block's attention must be done with the buffers
+                if (!claimed && nb > 0 &&
+                    !wait_bar(smem_u32(&bars->qk_free), (uint32_t)(nb - 1) & 1, abort_flag, wait_ns, p.status)) {
                     ok = false;
                     break;
                 }
-                if (warp == kEpi0 && lane == 0)
-                    QKV_TRACE_AT(2, n, 5 * x + 3);
-                if (r < NBr)
-                    epi_store(pv, smem + p.v_off + (size_t)r * kRowBytes, r);
+                if (mine) {
+                    epi_store(pq, smem + (size_t)r * kRowBytes, r);
+                    epi_store(pk, smem + p.k_off + (size_t)r * kRowBytes, r);
+                }
+                // V buffer nb & 1: the block two before must be done with it
+                const uint32_t vb = (uint32_t)nb & 1;
+                if (!claimed && nb > 1 &&
+                    !wait_bar(smem_u32(&bars->v_free[vb]), (uint32_t)((nb >> 1) - 1) & 1, abort_flag, wait_ns,
+                              p.status)) {
+                    ok = false;
+                    break;
+                }
+                claimed = true;
+                uint8_t *vbuf = smem + p.v_off + vb * p.v_size;
+                if (mine)
+                    epi_store(pv, vbuf + (size_t)r * kRowBytes, r);
+                if (cb.f0 + cb.L > td.f0 + kPTile)
+                    break;   // the block goes on in the next tile
+                // complete: clear V rows L..ceil16(L)-1, hand the block over
+                const int zr = cb.L + qq * 32 + lane;
+                if (zr < ((cb.L + 15) & ~15)) {
+                    uint4 *z = reinterpret_cast<uint4 *>(vbuf + (size_t)zr * kRowBytes);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        z[c] = make_uint4(0u, 0u, 0u, 0u);
+                }
                 fence_proxy_async_smem();   // the rows are read by the async proxy (MMAs)
                 __syncwarp();
-                if (lane == 0 && x == tiles - 1)
+                if (lane == 0)
                     mbar_arrive(smem_u32(&bars->qkv_ready));
-                if (warp == kEpi0 && lane == 0)
-                    QKV_TRACE_AT(2, n, 5 * x + 4);
-                ++tiles_done;
+                ++nb;
+                have = false;
             }
             if (!ok)
                 break;
@@ -498,15 +545,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t uses = 0;
         bool ok = true;
 
-        // Next unit: row tile 1 of the item if it has one, else row tile 0
-        // of the next item; the leader issues the unit's S MMA once the
-        // previous unit's O has been read and, for a new item, its Q, K and
+        // Next unit: row tile 1 of the block if it has one, else row tile 0
+        // of the next block; the leader issues the unit's S MMA once the
+        // previous unit's O has been read and, for a new block, its Q, K and
         // V are in shared memory.
         auto advance = [&]() -> bool {
             if (!(x == 0 && L > kQTile)) {
                 ++n;
-                ItemDesc d;
-                if (!read_desc(n, d)) {
+                Desc d;
+                if (!read_ring(bars->blk_full, bars->blk_empty, bars->blk, n, d)) {
                     ok = false;
                     return false;
                 }
@@ -530,19 +577,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     return false;
                 }
                 tc_fence_after();
-                if (lane == 0)
-                    QKV_TRACE_AT(3, n, 4 * x);
-                // A = Q of the row tile from TMEM (K = 64 in 4 steps of 8
-                // columns of bf16 pairs), B = K from shared memory
-                const uint32_t qa = tmem + kQCol + (uint32_t)(32 * x);
+                // A = Q rows of the row tile, B = K, both from shared memory
+                const uint64_t da = smem_desc_sw128(q_base + (uint32_t)(x * kQTile * kRowBytes), 16, 1024);
                 const uint64_t db = smem_desc_sw128(k_base, 16, 1024);
                 const uint32_t id_s = idesc_bf16_f32(128, nkeys, false);
                 if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(slot, qa + 8 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
+                        mma_ss(slot, da + 2 * kk, db + 2 * kk, id_s, kk > 0 ? 1u : 0u);
                     mma_commit(smem_u32(&bars->s_full));
-                    if (x == 1 || L <= kQTile)   // the item's last S: Q and K may be overwritten
+                    if (x == 1 || L <= kQTile)   // the block's last S: Q and K may be overwritten
                         mma_commit(smem_u32(&bars->qk_free));
                 }
                 __syncwarp();
@@ -583,15 +627,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(smem_u32(&bars->wg_p));
-            if (leader && lane == 0)
-                QKV_TRACE_AT(3, n, 4 * x + 1);
             // ---------------------------------------------- O = P V
             if (leader) {
                 if (!wait_bar(smem_u32(&bars->wg_p), uses & 1, abort_flag, wait_ns, p.status))
                     break;
                 tc_fence_after();
-                // V rows L..nkeys-1 are zeros (written so by the epilogue)
-                const uint64_t dv = smem_desc_sw128(v_base, 0, 1024);
+                // V rows L..nkeys-1 are zeros (cleared by the epilogue)
+                const uint64_t dv = smem_desc_sw128(v_base + ((uint32_t)n & 1) * p.v_size, 0, 1024);
                 if (lane == 0) {
                     const int ksteps = nkeys / 16;
 #pragma unroll
@@ -600,9 +642,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mma_ts(slot + kOCol, slot + kk * 8, dv + (uint64_t)(kk * (16 * kRowBytes >> 4)), id_pv,
                                    kk > 0 ? 1u : 0u);
                     mma_commit(smem_u32(&bars->o_full));
-                    QKV_TRACE_AT(3, n, 4 * x + 2);
-                    if (x == 1 || L <= kQTile)   // the item's last PV: V may be overwritten
-                        mma_commit(smem_u32(&bars->v_free));
+                    if (x == 1 || L <= kQTile)   // the block's last PV: its V buffer may be overwritten
+                        mma_commit(smem_u32(&bars->v_free[n & 1]));
                 }
                 __syncwarp();
             }
@@ -627,8 +668,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(smem_u32(&bars->wg_o));
-            if (leader && lane == 0)
-                QKV_TRACE_AT(3, n, 4 * x + 3);
             ++uses;
             pending = active;
             ef0 = f0;
@@ -653,7 +692,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tmem, kTmemCols);
     }
 }
-
 using QkvKernel = void (*)(CUtensorMap, CUtensorMap, Params);
 
 template <int NB>
@@ -724,11 +762,16 @@ extern "C" int nle_block_attn_qkv_fwd_ex(const void *x, const void *w_qkv, const
     p.heads = heads;
     p.B = B;
     p.ksteps = d_model / 64;
-    // shared memory: K and V of the item (NB rows each), the stage ring,
-    // the barriers; Q lives in TMEM
+    // shared memory: Q (NB rows, at least the 128 an S MMA reads; the S MMA
+    // of row tile 1 reads rows up to 255, past NB into K, whose results
+    // belong to rows past the block end and are never written), K (NB rows),
+    // two V buffers (NB rows each), the stage ring, the barriers
+    const uint32_t q_bytes = (uint32_t)(NB > kQTile ? NB : kQTile) * kRowBytes;
     const uint32_t kv_bytes = (uint32_t)NB * kRowBytes;
-    p.v_off = kv_bytes;
-    p.st_off = (2 * kv_bytes + 1023) & ~1023u;
+    p.k_off = q_bytes;
+    p.v_off = q_bytes + kv_bytes;
+    p.v_size = kv_bytes;
+    p.st_off = (q_bytes + 3 * kv_bytes + 1023) & ~1023u;
     const size_t bars_round = ((sizeof(Bars) + 127) / 128) * 128;
     int nst = 0;
     for (int s = kMaxStages; s >= 2; --s)

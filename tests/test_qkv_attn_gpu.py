@@ -81,6 +81,24 @@ def test_ragged_full_parity(lengths, heads, d_model, bias, cuda_device):
     _compare(_run(a, cuda_device), _ref(a))
 
 
+@pytest.mark.parametrize("seed", range(10))
+def test_random_batches(seed, cuda_device):
+    """Seeded random batches: many short utterances (a projection tile of 128
+    frames then holds many blocks, some of them a frame long) mixed with long
+    ones, block lengths from 16 to 256, 1 to 4 heads, d_model 64 to 256,
+    with and without a bias."""
+    rng = np.random.default_rng(900 + seed)
+    B = int(rng.choice([16, 64, 100, 129, 200, 256]))
+    n = int(rng.integers(1, 40))
+    lengths = [int(x) for x in rng.choice([0, 1, 2, 3, 7, 15, 64, 127, 128, 129, 200, 257, 600], n)]
+    if sum(lengths) == 0:
+        lengths[0] = 5
+    heads = int(rng.integers(1, 5))
+    d_model = int(rng.choice([64, 128, 192, 256]))
+    a = _inputs(lengths, heads, d_model, seed=1000 + seed, bias=bool(seed % 2))
+    _compare(_run(a, cuda_device, B=B), _ref(a, B=B))
+
+
 def test_encoder_shape_batch_slice(cuda_device):
     """The encoder's shape (d_model 1024, 16 heads) on 24 utterances of the
     batch-128 workload, with a bias."""
